@@ -1,0 +1,422 @@
+#!/usr/bin/env python3
+"""Benchmark of the Shannonic INT8 codec hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input resident in HBM:
+histogram → range DP + tANS tables → encode → decode (four C-ABI calls into libshn.so).
+Default workload: the INT8 KV cache [32 layers, K/V, batch 8, 8 kv heads, seq 4096, head_dim 128]
+(2 GiB, one table per layer×K/V), K=16, L=128, 4096-symbol chunks, 4 states per chunk.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload kv|weight|sweep]
+
+Multi-GPU (torchrun): every rank codes its own KV cache (seeded by rank) with no data-path
+collective — weak scaling; the time is the max over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from entropy_coded_lossless_b200 import inputs  # noqa: E402
+
+METRIC = "tANS decode/encode GB/s (INT8 side), % of HBM roofline; bits/symbol vs H"
+UNIT = "GB/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="kv", choices=["kv", "weight", "sweep", "activations"])
+    ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload(name, device, seed_offset=0):
+    """(int8 tensor, segments, params dict, description)."""
+    if name == "kv":
+        x = inputs.kv_cache_int8(seed=2 + seed_offset, device=device)
+        segs = inputs.kv_cache_segments()
+        desc = "kv_cache_int8[32,2,8,8,4096,128] (2 GiB, 64 segments = layer x K/V)"
+    elif name == "weight":
+        x = inputs.weight_like_int8(seed=1 + seed_offset, device=device)
+        segs = [(0, x.numel())]
+        desc = "weight_like_int8[4096,1024] (per-row absmax, 1% outliers x8)"
+    elif name == "activations":
+        x, segs, _ = inputs.activation_batch_int8(1024, 65536, seed=3 + seed_offset, device=device)
+        desc = "1024 activation tensors x 65536 INT8 (per-tensor tables)"
+    else:
+        x = inputs.sweep_stream_int8(5.3, seed=4 + seed_offset, device=device)
+        segs = [(0, x.numel())]
+        desc = "1 GiB truncated discrete Laplace, H=5.3 bits"
+    return x, segs, dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4), desc
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def stream_rate(stream_np, segs, p, hist):
+    """RP (payload bits/symbol), total bits/symbol and H from the stream and histograms (host, fp64)."""
+    hdr = np.frombuffer(stream_np[:64].tobytes(), dtype="<u8")
+    index_off, payload_off = int(hdr[5]), int(hdr[6])
+    n_segs = len(segs)
+    descs = np.frombuffer(stream_np[64:64 + 32 * n_segs].tobytes(), dtype="<u4").reshape(n_segs, 8)
+    total_chunks = int(hdr[4])
+    index = np.frombuffer(stream_np[index_off:index_off + 4 * total_chunks].tobytes(), dtype="<u4").astype(np.int64)
+    words = np.frombuffer(stream_np[payload_off:].tobytes()[: (len(stream_np) - payload_off) // 4 * 4], dtype="<u4")
+    payload_bits = 0
+    for s in range(n_segs):
+        first = int(descs[s, 7])
+        nch = -(-segs[s][1] // p["chunk_symbols"])
+        start_w = int(descs[s, 4] | (descs[s, 5] << 32)) // 4
+        pay_words = int(descs[s, 6])
+        if nch == 0:
+            continue
+        ends = np.append(index[first + 1:first + nch], pay_words)
+        last = words[start_w + ends - 1].astype(np.int64)
+        hb = np.floor(np.log2(np.maximum(last, 1))).astype(np.int64)
+        T = 32 * (ends - 1) + hb  # sentinel position = bits before it
+        T -= 32 * np.append(0, ends[:-1])
+        payload_bits += int(T.sum()) - nch * p["states_per_chunk"] * p["log2L"]
+    n = sum(l for _, l in segs)
+    h = hist.reshape(-1, 256).astype(np.float64)
+    ent = 0.0
+    for s in range(n_segs):
+        row = h[s]
+        tot = row.sum()
+        if tot > 0:
+            q = row[row > 0] / tot
+            ent += float(-(q * np.log2(q)).sum()) * tot
+    H = ent / n
+    rp = payload_bits / n
+    return {"payload": rp, "total": 8.0 * len(stream_np) / n, "entropy": H, "diff_pct": (rp - H) / H * 100.0}
+
+
+def cpu_baseline(x_dev, segs, p, budget_s, full_n):
+    """The CPU oracle as it stands (encode + decode, all host threads) on a bounded sample of the
+    same workload: whole segments, as many as fit the time budget (at least one)."""
+    import oracle
+
+    cores = oracle.cpu_count()
+    o0, n0 = segs[0]
+    one = x_dev[o0:o0 + n0].cpu().numpy()
+    t = time.perf_counter()
+    s, _ = oracle.encode(one, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], threads=cores)
+    rc, _ = oracle.decode(s, threads=cores)
+    dt1 = time.perf_counter() - t
+    k = max(1, min(len(segs), int(budget_s / max(dt1, 1e-3))))
+    sample = [segs[i] for i in range(k)]
+    xs = np.concatenate([x_dev[o:o + n].cpu().numpy() for o, n in sample])
+    local = []
+    off = 0
+    for _, n in sample:
+        local.append((off, n))
+        off += n
+    t = time.perf_counter()
+    s, _ = oracle.encode(xs, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], segments=local,
+                         threads=cores)
+    rc, y = oracle.decode(s, threads=cores)
+    dt = time.perf_counter() - t
+    assert rc == 0 and np.array_equal(y, xs.view(np.uint8))
+    nbytes = xs.size
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{k} of {len(segs)} segments ({nbytes} bytes): histogram+DP+tables+encode+decode, "
+                      f"{dt:.1f} s on {cores} host threads"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x, segs, p, desc = workload(args.workload, "cpu")
+    import oracle
+
+    cores = oracle.cpu_count()
+    # each step: a bounded sample (whole segments) of the workload, histogram → tables → encode → decode
+    o0, n0 = segs[0]
+    one = x[o0:o0 + n0].numpy()
+    t = time.perf_counter()
+    s, _ = oracle.encode(one, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], threads=cores)
+    oracle.decode(s, threads=cores)
+    dt1 = time.perf_counter() - t
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    k = max(1, min(len(segs), int(per_step_budget / max(dt1, 1e-3))))
+    sample = segs[:k]
+    xs = np.concatenate([x[o:o + n].numpy() for o, n in sample])
+    local, off = [], 0
+    for _, n in sample:
+        local.append((off, n))
+        off += n
+
+    def step():
+        s, _ = oracle.encode(xs, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], segments=local,
+                             threads=cores)
+        rc, y = oracle.decode(s, threads=cores)
+        assert rc == 0
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t) / args.steps
+    v = xs.size / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": desc, "K": p["K"], "L": 1 << p["log2L"], "chunk_symbols": p["chunk_symbols"],
+                       "states_per_chunk": p["states_per_chunk"], "sample_segments": k},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{k} of {len(segs)} segments per step ({xs.size} bytes)"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    from entropy_coded_lossless_b200 import shn
+
+    x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank)
+    p = shn.CodecParams(**p_dict)
+    codec = shn.Codec(segs, p, device=dev)
+    n = codec.n_symbols
+    out = torch.empty(n, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    comp_cap = codec.stream_buf.numel()
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    stage_ms = {"histogram": 0.0, "build": 0.0, "encode": 0.0, "decode": 0.0}
+
+    def step(timed):
+        if timed:
+            ev[0].record(stream)
+        codec.histogram(x)
+        if timed:
+            ev[1].record(stream)
+        codec.build()
+        if timed:
+            ev[2].record(stream)
+        codec.encode(x)
+        if timed:
+            ev[3].record(stream)
+        codec.decode(codec.stream_buf, comp_cap, out)
+        if timed:
+            ev[4].record(stream)
+            ev[4].synchronize()
+            for i, k in enumerate(stage_ms):
+                stage_ms[k] += ev[i].elapsed_time(ev[i + 1])
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+
+    # correctness of the timed work
+    est, edet = codec.status("enc")
+    dst, ddet = codec.status("dec")
+    ok = est == 0 and dst == 0 and torch.equal(out, x.view(torch.uint8))
+    nbytes = int(codec.out_bytes.item())
+    stream_np = codec.stream_buf[:nbytes].cpu().numpy()
+    rate = stream_rate(stream_np, segs, p_dict, codec.hist.cpu().numpy())
+
+    # e2e through the C ABI with host buffers: pinned H2D of the input, the four calls, D2H of the stream
+    e2e = None
+    if not args.no_e2e:
+        h_in = torch.empty(n, dtype=torch.int8, pin_memory=True)
+        h_in.copy_(x.cpu())
+        h_out = torch.empty(comp_cap, dtype=torch.uint8, pin_memory=True)
+        h_st = torch.empty(16, dtype=torch.uint8, pin_memory=True)
+        x_e = torch.empty_like(x)
+
+        def e2e_step():
+            x_e.copy_(h_in, non_blocking=True)
+            codec.histogram(x_e)
+            codec.build()
+            codec.encode(x_e)
+            codec.decode(codec.stream_buf, comp_cap, out)
+            h_out[:nbytes].copy_(codec.stream_buf[:nbytes], non_blocking=True)
+            h_st[:8].copy_(codec.work_enc[:8], non_blocking=True)
+            h_st[8:16].copy_(codec.work_dec[:8], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ksteps = max(1, min(args.steps, 3))
+        e0.record(stream)
+        for _ in range(ksteps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1) / ksteps
+        if world > 1:
+            tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(tt.item())
+        e2e = {"value": world * n / (ms_e2e * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": n,
+               "d2h_bytes_per_step": nbytes + 16, "ms_per_step": ms_e2e,
+               "what": "pinned H2D input + shn_histogram + shn_build_tables + shn_encode + shn_decode + D2H stream/status"}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        stages = {}
+        for k, v in stage_ms.items():
+            ms = v / args.steps
+            stages[k] = {"ms": ms, "gbs_int8": n / (ms * 1e-3) / 1e9 if ms > 0 else None}
+        alg = {"histogram": n, "build": 0, "encode": n + nbytes, "decode": n + nbytes}
+        dom = max(("encode", "decode", "histogram"), key=lambda k: stages[k]["ms"])
+
+        def roof(k):
+            ms = stages[k]["ms"]
+            a = alg[k] / (ms * 1e-3) / 1e9
+            return {"bound": "hbm", "achieved": a, "peak": peak, "unit": "GB/s", "frac": a / peak,
+                    "traffic": None, "kernel": {"decode": "decode_kernel", "encode": "encode_{sizes,write}_kernel",
+                                                "histogram": "histogram_kernel"}[k],
+                    "alg_bytes_per_launch": alg[k], "peak_kind": peak_kind}
+
+        launches_per_step = 1 + 1 + 1 + 3 + 1 + 1 + 2  # hist, build, sizes, scan x3, header, write, check+decode
+        line = {
+            "metric": METRIC,
+            "value": world * n / (ms_step * 1e-3) / 1e9,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "u8",
+            "data": "synthetic",
+            "config": {"workload": desc, "K": p.K, "L": 1 << p.log2L, "chunk_symbols": p.chunk_symbols,
+                       "states_per_chunk": p.states_per_chunk, "bytes_per_gpu": n,
+                       "l2": "inputs larger than L2 (2 GiB in, ~1.9 GB stream, 2 GiB out per step)"
+                       if n > (1 << 28) else "input smaller than L2; no flush",
+                       "parallelism": f"replicas x{world} (independent segments per rank)"},
+            "step": "histogram + DP/tables + encode + decode (value = INT8 bytes per step / step time)",
+            "stages": stages,
+            "roofline": roof(dom),
+            "roofline_decode": roof("decode"),
+            "roofline_encode": roof("encode"),
+            "bits_per_symbol": rate,
+            "stream_bytes": nbytes,
+            "correct": bool(ok),
+            "clocks": clk.summary(),
+            "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(x, segs, p_dict, args.cpu_sample_seconds, n)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if not ok:
+        sys.exit(3)
+
+
+if __name__ == "__main__":
+    main()

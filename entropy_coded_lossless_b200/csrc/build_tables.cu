@@ -1,0 +1,289 @@
+// build_tables.cu — per-segment range selection and tANS tables, one block per table.
+//
+// Shannonic §4.1 (preprocessing): partition the 256-value alphabet into K contiguous ranges by the
+// DP C[i,k] = min_{j<i} { C[j,k-1] + Cost(j,i-1) } with backtracking from C[256,K]; derive the
+// per-range parameters (base, offset bits, encTable start, normalisation bias), rangeId[256], and an
+// L-entry tANS table from the range probabilities. The exact integer rules (fixed-point log2, cost,
+// tie-breaks, state-count allocation, spread) are FORMAT.md §2-§5; this kernel must reproduce them
+// bit for bit, so it uses only integer arithmetic.
+//
+// Work is tiny (O(K·256²/2) min-plus steps per table) and latency-bound; one block of 512 threads
+// per table keeps everything in shared memory: the fixed-point log2 of every range count (a
+// triangular 256x256 table), two DP rows and the K x 257 argmin matrix.
+#include "shn_internal.cuh"
+
+namespace shn {
+
+constexpr int kBuildThreads = 512;
+constexpr int kPairs = 256 * 257 / 2;  // ranges [j, i), 0 <= j < i <= 256
+
+__device__ __forceinline__ int pair_index(int j, int i) { return i * (i - 1) / 2 + j; }
+__device__ __forceinline__ uint32_t ceil_log2_width(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
+
+struct BuildShared {
+  uint32_t pre[257];       // prefix sums of the histogram (total < 2^32)
+  long long drow[2][257];  // DP rows D[.][k-1], D[.][k]
+  uint32_t lgf[4097];      // LG(f) for f = 0..L
+  uint32_t f[256];
+  uint32_t cumul[257];
+  uint32_t lo[257];
+  uint32_t rng[256];       // range of each symbol u
+  uint8_t spread[4096];
+  uint32_t status;
+  long long cost;
+};
+
+__global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsigned long long* __restrict__ hist_all,
+                                                                     shn_params p, shn_table* __restrict__ tables_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BuildShared& S = *reinterpret_cast<BuildShared*>(smem_raw);
+  uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));          // kPairs
+  uint8_t* arg = reinterpret_cast<uint8_t*>(lgc + kPairs);                               // K x 257
+
+  const int tid = threadIdx.x;
+  const int K = (int)p.K;
+  const int R = (int)p.log2L;
+  const uint32_t L = 1u << R;
+  const unsigned long long* hist = hist_all + (size_t)blockIdx.x * 256;
+  shn_table* out = tables_out + blockIdx.x;
+
+  // ---- prefix sums and the 2^32 bound --------------------------------------------------------
+  if (tid == 0) {
+    unsigned long long acc = 0;
+    S.pre[0] = 0;
+    for (int u = 0; u < 256; ++u) {
+      acc += hist[u];
+      S.pre[u + 1] = (uint32_t)acc;
+    }
+    S.status = acc >= (1ull << 32) ? (uint32_t)SHN_ERR_INVALID_ARG : 0u;
+    S.cost = 0;
+    out->n = acc;
+  }
+  for (uint32_t f = tid; f <= L; f += kBuildThreads) S.lgf[f] = lg_fixed(f);
+  __syncthreads();
+  if (S.status != 0) {
+    if (tid == 0) {
+      out->K = K;
+      out->log2L = R;
+      out->status = S.status;
+    }
+    return;
+  }
+
+  // ---- range selection (FORMAT.md §3) ---------------------------------------------------------
+  if (K == 256) {
+    if (tid < 256) S.lo[tid] = tid;
+    if (tid == 0) {
+      long long c = 0;
+      for (int u = 0; u < 256; ++u) {
+        const uint32_t n = S.pre[u + 1] - S.pre[u];
+        c -= (long long)n * lg_fixed(n);
+      }
+      S.cost = c;
+    }
+  } else {
+    for (int q = tid; q < kPairs; q += kBuildThreads) {
+      int i = (int)((1.0f + sqrtf(8.0f * (float)q + 1.0f)) * 0.5f);
+      while (i * (i - 1) / 2 > q) --i;
+      while ((i + 1) * i / 2 <= q) ++i;
+      const int j = q - i * (i - 1) / 2;
+      lgc[q] = lg_fixed(S.pre[i] - S.pre[j]);
+    }
+    for (int i = tid; i <= 256; i += kBuildThreads) S.drow[0][i] = (i == 0) ? 0 : LLONG_MAX;
+    __syncthreads();
+    // two lanes per end point i: lane parity h takes j = jmin + h, jmin + h + 2, ...
+    const int h = tid & 1;
+    const int i = 256 - (tid >> 1);  // 256 .. 1
+    for (int k = 1; k <= K; ++k) {
+      const long long* prev = S.drow[(k - 1) & 1];
+      long long* cur = S.drow[k & 1];
+      long long best = LLONG_MAX;
+      int bj = 0x7fffffff;
+      if (i >= k) {
+        const int jmax = (k == 1) ? 0 : i - 1;
+        const uint32_t pi = S.pre[i];
+        for (int j = k - 1 + h; j <= jmax; j += 2) {
+          const uint32_t c = pi - S.pre[j];
+          const long long w = (long long)ceil_log2_width((uint32_t)(i - j));
+          const long long cost = (long long)c * (w << 24) - (long long)((unsigned long long)c * lgc[pair_index(j, i)]);
+          const long long v = prev[j] + cost;
+          if (v < best) {
+            best = v;
+            bj = j;
+          }
+        }
+      }
+      const long long ob = __shfl_xor_sync(0xffffffffu, best, 1);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, 1);
+      if (ob < best || (ob == best && oj < bj)) {
+        best = ob;
+        bj = oj;
+      }
+      if (h == 0) {
+        if (i >= k) {
+          cur[i] = best;
+          arg[(size_t)(k - 1) * 257 + i] = (uint8_t)bj;
+        }
+      }
+      if (tid == 0) cur[0] = LLONG_MAX;
+      if (tid < 257 && tid < k) cur[tid] = LLONG_MAX;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      S.cost = S.drow[K & 1][256];
+      int ii = 256;
+      for (int k = K; k >= 1; --k) {
+        const int j = arg[(size_t)(k - 1) * 257 + ii];
+        S.lo[k - 1] = (uint32_t)j;
+        ii = j;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) S.lo[K] = 256;
+  __syncthreads();
+
+  // ---- state counts (FORMAT.md §4): one warp, greedy with smallest-k tie-break ---------------
+  if (tid < 32) {
+    constexpr int kPer = 8;  // ranges per lane (K <= 256)
+    unsigned long long N[kPer];
+    uint32_t f[kPer];
+    int nonzero = 0;
+    unsigned long long total = 0;
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int k = tid + 32 * r;
+      N[r] = (k < K) ? (unsigned long long)(S.pre[S.lo[k + 1]] - S.pre[S.lo[k]]) : 0ull;
+      f[r] = N[r] > 0 ? 1u : 0u;
+      nonzero += (int)f[r];
+      total += N[r];
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      nonzero += __shfl_xor_sync(0xffffffffu, nonzero, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    if (total == 0) {
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) f[r] = (tid == 0 && r == 0) ? L : 0u;
+    } else {
+      // K <= L is checked on the host, so nonzero <= L
+      for (uint32_t step = 0; step < L - (uint32_t)nonzero; ++step) {
+        unsigned long long bg = 0;
+        int bk = 0x7fffffff;
+#pragma unroll
+        for (int r = 0; r < kPer; ++r) {
+          const int k = tid + 32 * r;
+          if (N[r] > 0) {
+            const unsigned long long g = N[r] * (unsigned long long)(S.lgf[f[r] + 1] - S.lgf[f[r]]);
+            if (bk == 0x7fffffff || g > bg || (g == bg && k < bk)) {
+              bg = g;
+              bk = k;
+            }
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long og = __shfl_xor_sync(0xffffffffu, bg, o);
+          const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
+          if (ok != 0x7fffffff && (bk == 0x7fffffff || og > bg || (og == bg && ok < bk))) {
+            bg = og;
+            bk = ok;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < kPer; ++r)
+          if (tid + 32 * r == bk) f[r] += 1;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int k = tid + 32 * r;
+      if (k < 256) S.f[k] = (k < K) ? f[r] : 0u;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t acc = 0;
+    for (int k = 0; k < K; ++k) {
+      S.cumul[k] = acc;
+      acc += S.f[k];
+    }
+    S.cumul[K] = acc;
+  }
+  if (tid < 256) {
+    // range of symbol u: largest k with lo[k] <= u
+    int a = 0, b2 = K - 1;
+    while (a < b2) {
+      const int m = (a + b2 + 1) >> 1;
+      if (S.lo[m] <= (uint32_t)tid) a = m;
+      else b2 = m - 1;
+    }
+    S.rng[tid] = (uint32_t)a;
+  }
+  __syncthreads();
+
+  // ---- spread (FORMAT.md §5) ------------------------------------------------------------------
+  const uint32_t step = (L >> 1) + (L >> 3) + 3;
+  for (uint32_t t = tid; t < L; t += kBuildThreads) {
+    int a = 0, b2 = K - 1;  // largest k with cumul[k] <= t
+    while (a < b2) {
+      const int m = (a + b2 + 1) >> 1;
+      if (S.cumul[m] <= t) a = m;
+      else b2 = m - 1;
+    }
+    S.spread[(t * step) & (L - 1)] = (uint8_t)a;
+  }
+  __syncthreads();
+
+  // ---- encode table: enc[cumul_s + j] = L + (j-th slot of s) ---------------------------------
+  uint16_t* enc = reinterpret_cast<uint16_t*>(out->opaque + kOpaqueEncOffset);
+  for (int k = tid; k < K; k += kBuildThreads) {
+    uint32_t j = S.cumul[k];
+    if (S.f[k] == 0) continue;
+    for (uint32_t i = 0; i < L; ++i)
+      if (S.spread[i] == (uint8_t)k) enc[j++] = (uint16_t)(L + i);
+  }
+  // ---- per raw byte encoder entries -----------------------------------------------------------
+  if (tid < 256) {
+    const uint32_t bb = (uint32_t)tid;  // raw byte
+    const uint32_t u = bb ^ 0x80u;
+    const uint32_t s = S.rng[u];
+    const uint32_t fs = S.f[s];
+    const uint32_t o = u - S.lo[s];
+    const uint32_t w = ceil_log2_width(S.lo[s + 1] - S.lo[s]);
+    uint2 e;
+    if (fs == 0) {
+      e.x = 0u;  // nb = 0; enc index = X - L stays inside the table
+      e.y = (4096u - L) | (o << 16) | (w << 24) | 0x80000000u;  // absent-symbol flag
+    } else {
+      const uint32_t a = 31u - __clz(fs);
+      const uint32_t sh = (uint32_t)R - a;
+      e.x = (sh << 16) - (fs << sh);
+      e.y = (uint32_t)((int)S.cumul[s] - (int)fs + 4096) | (o << 16) | (w << 24);
+    }
+    reinterpret_cast<uint2*>(out->opaque + kOpaqueSymOffset)[bb] = e;
+    out->f[tid] = (uint16_t)S.f[tid];
+    out->lo[tid] = (uint8_t)((tid < K) ? S.lo[tid] : 0u);
+  }
+  if (tid == 0) {
+    uint32_t wmax = 0;
+    for (int k = 0; k < K; ++k) wmax = max(wmax, ceil_log2_width(S.lo[k + 1] - S.lo[k]));
+    out->K = K;
+    out->log2L = R;
+    out->status = 0;
+    out->w_max = wmax;
+    out->dp_cost = S.cost;
+  }
+}
+
+cudaError_t launch_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params& p, shn_table* d_tables,
+                                cudaStream_t s) {
+  if (n_tables == 0) return cudaSuccess;
+  const size_t smem = sizeof(BuildShared) + sizeof(uint32_t) * kPairs + (size_t)p.K * 257;
+  cudaError_t e = cudaFuncSetAttribute(build_tables_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  build_tables_kernel<<<n_tables, kBuildThreads, smem, s>>>(reinterpret_cast<const unsigned long long*>(d_hist), p,
+                                                            d_tables);
+  return cudaGetLastError();
+}
+
+}  // namespace shn

@@ -1,0 +1,143 @@
+// shn_internal.cuh — internal definitions shared by the libshn kernels and the C-ABI layer.
+//
+// The SHN1 stream layout and every table rule are those of FORMAT.md (the codec's bitstream
+// specification), which restates the Shannonic method ("Shannonic: Efficient Entropy-Optimal
+// Compression for ML Workloads", MLSys 2026 notes, §4.1 preprocessing and §4.2 Algorithm 2).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/shn.h"
+
+namespace shn {
+
+// ---- stream layout (FORMAT.md §6) -------------------------------------------------------------
+constexpr uint32_t kMagic = 0x314E4853u;  // "SHN1"
+constexpr uint32_t kHeaderBytes = 64;
+constexpr uint32_t kSegDescBytes = 32;
+
+__host__ __device__ inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline uint32_t table_record_bytes(uint32_t K) { return (uint32_t)round_up(3ull * K, 4); }
+__host__ __device__ inline uint64_t index_offset(uint32_t n_segs, uint32_t K) {
+  return kHeaderBytes + (uint64_t)kSegDescBytes * n_segs + (uint64_t)table_record_bytes(K) * n_segs;
+}
+__host__ __device__ inline uint64_t payload_offset(uint32_t n_segs, uint32_t K, uint64_t total_chunks) {
+  return round_up(index_offset(n_segs, K) + 4ull * total_chunks, 16);
+}
+__host__ __device__ inline uint64_t n_chunks(uint64_t n, uint32_t C) { return (n + C - 1) / C; }
+// Words of a chunk of c symbols in the worst case: S states + c fields of <= R+8 bits + sentinel.
+__host__ __device__ inline uint64_t chunk_max_words(uint32_t S, uint32_t R, uint64_t c) {
+  return ((uint64_t)S * R + c * (uint64_t)(R + 8) + 1 + 31) / 32;
+}
+
+// ---- device table record (include/shn.h: shn_table) -----------------------------------------
+// opaque part: uint2 sym[256] for every raw byte b (u = b ^ 0x80):
+//   .x = bias[s]  (nb = (X + bias) >> 16),
+//   .y = (start[s] + 4096) | (offset << 16) | (w << 24)   with start[s] = cumul_s - f_s,
+// then uint16 enc[L] holding the next state L + slot.
+constexpr uint32_t kOpaqueSymOffset = 0;
+constexpr uint32_t kOpaqueEncOffset = 2048;
+static_assert(sizeof(shn_table) == SHN_TABLE_BYTES, "table record size");
+static_assert(offsetof(shn_table, opaque) == SHN_TABLE_PUBLIC_BYTES, "table public size");
+
+__device__ __forceinline__ const uint2* table_sym(const shn_table* t) {
+  return reinterpret_cast<const uint2*>(t->opaque + kOpaqueSymOffset);
+}
+__device__ __forceinline__ const uint16_t* table_enc(const shn_table* t) {
+  return reinterpret_cast<const uint16_t*>(t->opaque + kOpaqueEncOffset);
+}
+
+// ---- device status word (first 8 bytes of every workspace) -----------------------------------
+struct DeviceStatus {
+  uint32_t status;
+  uint32_t detail;
+};
+
+__device__ __forceinline__ void report(DeviceStatus* st, uint32_t code, uint32_t detail) {
+  if (atomicCAS(&st->status, 0u, code) == 0u) st->detail = detail;
+}
+
+// ---- FORMAT.md §2 fixed-point log2: 24 fraction bits by repeated squaring -------------------
+__device__ __forceinline__ uint32_t lg_fixed(uint32_t n) {
+  if (n == 0) return 0;
+  const int e = 31 - __clz(n);
+  unsigned long long m = (unsigned long long)n << (31 - e);
+  uint32_t frac = 0;
+#pragma unroll
+  for (int it = 0; it < 24; ++it) {
+    m = (m * m) >> 31;
+    const uint32_t bit = (uint32_t)(m >> 32);  // 1 iff m >= 2^32 (m < 2^33)
+    frac = (frac << 1) | bit;
+    m >>= bit;
+  }
+  return ((uint32_t)e << 24) | frac;
+}
+
+// ---- segment batches passed by value to kernels (no device allocation) ---------------------
+constexpr int kSegBatch = 512;
+
+struct HistBatch {
+  uint32_t n;                      // segments in this batch
+  uint32_t total_blocks;           // blocks of the launch
+  uint64_t offset[kSegBatch];      // byte offset in d_in
+  uint32_t length[kSegBatch];      // bytes
+  uint32_t block_start[kSegBatch]; // first block of each segment
+  uint32_t hist_index[kSegBatch];  // histogram row of each segment
+};
+
+struct EncBatch {
+  uint32_t n;
+  uint32_t total_blocks;
+  uint64_t offset[kSegBatch];      // byte offset in d_in
+  uint64_t out_offset[kSegBatch];  // sum of the lengths of all earlier segments
+  uint32_t length[kSegBatch];
+  uint32_t first_chunk[kSegBatch]; // global chunk index
+  uint32_t block_start[kSegBatch];
+  uint32_t seg_index[kSegBatch];   // segment / table index
+};
+
+// Launch wrappers (defined in the .cu files; return a cudaError_t).
+cudaError_t launch_histogram(const uint8_t* d_in, const HistBatch& b, uint64_t* d_hist, int threads,
+                             cudaStream_t s);
+uint32_t histogram_blocks_for(uint64_t length);
+cudaError_t launch_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params& p,
+                                shn_table* d_tables, cudaStream_t s);
+
+struct EncodeLayout {
+  uint32_t n_segs;
+  uint32_t K, R, S, C;
+  uint64_t total_chunks;
+  uint64_t total_symbols;
+  uint64_t index_offset;
+  uint64_t payload_offset;
+  uint64_t out_capacity;
+};
+
+// Workspace layout of shn_encode: [status 256 B][chunk words u32 x total_chunks, padded]
+// [global word offsets u64 x (total_chunks+1)][block partial sums u64 x n_blocks+1]
+struct EncodeWork {
+  DeviceStatus* status;
+  uint32_t* chunk_words;
+  unsigned long long* word_offset;  // exclusive prefix over all chunks, total at [total_chunks]
+  unsigned long long* block_sums;
+  uint32_t scan_blocks;
+};
+constexpr uint32_t kScanBlock = 1024;  // chunks reduced per scan block
+
+cudaError_t launch_encode_sizes(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
+                                const EncodeLayout& lay, const EncodeWork& w, int threads, cudaStream_t s);
+cudaError_t launch_scan(const EncodeWork& w, uint64_t total_chunks, cudaStream_t s);
+cudaError_t launch_encode_header(const EncBatch& b, const shn_table* d_tables, const EncodeLayout& lay,
+                                 const EncodeWork& w, uint8_t* d_out, uint64_t* d_out_bytes, bool first_batch,
+                                 cudaStream_t s);
+cudaError_t launch_encode_empty(const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, uint64_t* d_out_bytes,
+                                cudaStream_t s);
+cudaError_t launch_encode_write(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
+                                const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, int threads,
+                                cudaStream_t s);
+
+cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
+                          uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s);
+
+}  // namespace shn

@@ -1,0 +1,176 @@
+/*
+ * shn.h — C ABI of the B200 Shannonic INT8 entropy codec (libshn.so).
+ *
+ * The codec is the Shannonic scheme of "Shannonic: Efficient Entropy-Optimal Compression for ML
+ * Workloads" (MLSys 2026 talk notes): a 256-bin histogram, a dynamic-programming split of the value
+ * space into K contiguous ranges, and tANS over the range indices with raw fixed-width offsets
+ * (§4, §4.1, §4.2 Algorithm 2). The bitstream ("SHN1") is fixed by FORMAT.md.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named d_* are CUDA device pointers, h_* are host pointers. All memory belongs to the
+ *    caller; the library never allocates device memory and never synchronises the device, except in
+ *    shn_get_device_status (documented below).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is enqueued
+ *    asynchronously on it and runs on the device that is current for the calling thread.
+ *  - Return value: an shn_status. Errors a host check can see (bad parameters, sizes, alignment,
+ *    too-small buffers computable on the host) are returned immediately and nothing is enqueued.
+ *    Errors only the device can see (a corrupt stream, an output larger than its buffer) are
+ *    written to the status word at the start of the caller's workspace (d_work); kernels then skip
+ *    the rest of their work and return normally — no trap, no hang. Read it with
+ *    shn_get_device_status or by copying the first 8 bytes of d_work.
+ *  - Symbols: byte b of an INT8 tensor is coded as u = b XOR 0x80 (signed value + 128).
+ */
+#ifndef SHN_H
+#define SHN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SHN_VERSION 0x00010000u /* 1.0.0; the stream format version is 1 */
+
+/* Size of one shn_table record in bytes (a multiple of 256). */
+#define SHN_TABLE_BYTES 11264u
+#define SHN_TABLE_PUBLIC_BYTES 800u
+
+typedef enum shn_status {
+  SHN_OK = 0,
+  SHN_ERR_INVALID_ARG = 1, /* bad parameter, pointer, size or alignment */
+  SHN_ERR_CAPACITY = 2,    /* an output buffer is too small */
+  SHN_ERR_CORRUPT = 3,     /* the compressed stream fails a structural or end-of-chunk check */
+  SHN_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+  SHN_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reserved; current kernels never wait) */
+  SHN_ERR_UNSUPPORTED = 6, /* valid parameters this build's kernels do not implement */
+  SHN_ERR_WORKSPACE = 7    /* the workspace is smaller than the *_workspace_bytes query returned */
+} shn_status;
+
+/* A segment is a run of input bytes coded with its own table (one tensor, one KV layer, …). */
+typedef struct shn_segment {
+  uint64_t offset; /* byte offset of the segment within d_in */
+  uint64_t length; /* number of INT8 values; must be < 2^32 */
+} shn_segment;
+
+/* Codec parameters (FORMAT.md §6 constraints). */
+typedef struct shn_params {
+  uint32_t K;                /* number of ranges, 1 <= K <= min(256, L); K = 256 is plain tANS */
+  uint32_t log2L;            /* R: tANS state count L = 2^R, 4 <= R <= 12 */
+  uint32_t chunk_symbols;    /* C: symbols per chunk, multiple of 128, 128 <= C <= 65536 */
+  uint32_t states_per_chunk; /* S: interleaved tANS states per chunk, one of 1, 2, 4, 8, 16 */
+} shn_params;
+
+/*
+ * Per-table device record written by shn_build_tables (SHN_TABLE_BYTES each, 256-byte aligned
+ * when d_tables is). The leading fields are public and stable; `opaque` holds the encoder's
+ * lookup tables and must not be modified.
+ */
+typedef struct shn_table {
+  uint32_t K;       /* ranges */
+  uint32_t log2L;   /* R */
+  uint32_t status;  /* SHN_OK, or SHN_ERR_INVALID_ARG when the histogram total is >= 2^32 */
+  uint32_t w_max;   /* largest offset field width over the ranges */
+  int64_t dp_cost;  /* D[256][K] of the range DP, units of 2^-24 bit (FORMAT.md §3) */
+  uint64_t n;       /* histogram total */
+  uint16_t f[256];  /* tANS state count of each range (sum = L); entries >= K are 0 */
+  uint8_t lo[256];  /* first symbol u of each range; range k = [lo[k], lo[k+1]) with lo[K] = 256 */
+  uint8_t opaque[SHN_TABLE_BYTES - SHN_TABLE_PUBLIC_BYTES];
+} shn_table;
+
+/* --- queries (host only, no CUDA calls) --------------------------------------------------- */
+
+uint32_t shn_version(void);
+const char* shn_status_string(int status);
+
+/* SHN_OK if p satisfies the FORMAT.md §6 constraints, else SHN_ERR_INVALID_ARG. */
+int shn_check_params(const shn_params* p);
+
+/* Bytes of one table record in d_tables (constant, = sizeof(shn_table)). */
+size_t shn_table_bytes(const shn_params* p);
+
+/* Largest SHN1 stream shn_encode can produce for these segments (0 on bad arguments). */
+size_t shn_encode_bound(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs);
+
+/* Device workspace shn_encode needs (per-chunk sizes and scan scratch + the status word). */
+size_t shn_encode_workspace_bytes(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs);
+
+/* Device workspace shn_decode needs (the status word only). */
+size_t shn_decode_workspace_bytes(const shn_params* p);
+
+/* --- the codec ---------------------------------------------------------------------------- */
+
+/*
+ * 256-bin histogram of each segment (Shannonic §4.1: "compute the histogram h[x] of the input
+ * tensor"). d_hist[s*256 + u] = number of bytes b in segment s with (b ^ 0x80) == u.
+ *  d_in    device, the input bytes; any alignment.
+ *  h_segs  host array of n_segs segments; every segment must lie inside d_in's allocation.
+ *  d_hist  device, n_segs*256 uint64, 8-byte aligned; fully overwritten.
+ * Errors: SHN_ERR_INVALID_ARG (NULL pointers with n_segs > 0, segment length >= 2^32),
+ *         SHN_ERR_CUDA.
+ */
+int shn_histogram(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, uint64_t* d_hist,
+                  void* stream);
+
+/*
+ * Range selection and tANS tables for each histogram (Shannonic §4.1: DP range selection
+ * C[i,k] = min_{j<i} C[j,k-1] + Cost(j,i-1) with backtracking from C[256,K]; per-range base,
+ * offset width, encTable start and bias; rangeId[256]; an L-state tANS table from the range
+ * probabilities). Exact rules: FORMAT.md §2-§5. One CUDA block per table.
+ *  d_hist    device, n_tables*256 uint64 (as written by shn_histogram).
+ *  d_tables  device, n_tables*shn_table_bytes(p) bytes, 256-byte aligned; fully overwritten.
+ * A histogram whose total is >= 2^32 gets status SHN_ERR_INVALID_ARG in its record (and makes
+ * shn_encode report SHN_ERR_INVALID_ARG on the device).
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_CUDA.
+ */
+int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params* p, void* d_tables,
+                     void* stream);
+
+/*
+ * Encode segments into one SHN1 stream (Shannonic §4.2, Algorithm 2: per value, s = rangeId[x],
+ * emit the offset x - base[s] in nb[s] bits, emit the state-normalisation bits, move the state
+ * through encTable). Chunks of C symbols are coded independently with S interleaved states.
+ *  d_in          device input bytes; every segment offset must be 16-byte aligned with d_in
+ *                16-byte aligned (SHN_ERR_INVALID_ARG otherwise).
+ *  h_segs        host, n_segs segments; segment s is coded with table s of d_tables.
+ *  d_tables      device, n_segs records from shn_build_tables with the same params.
+ *  d_work        device workspace of >= shn_encode_workspace_bytes(p, h_segs, n_segs) bytes,
+ *                256-byte aligned. Its first 8 bytes receive the device status.
+ *  d_out         device, out_capacity bytes, 16-byte aligned; receives the stream.
+ *  d_out_bytes   device uint64: the stream size in bytes (written even when it exceeds the
+ *                capacity, in which case the device status is SHN_ERR_CAPACITY and d_out holds
+ *                no complete stream).
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_WORKSPACE, SHN_ERR_CUDA; device: SHN_ERR_CAPACITY,
+ *         SHN_ERR_INVALID_ARG (a table with bad status or a symbol absent from its table).
+ */
+int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, const void* d_tables,
+               const shn_params* p, void* d_work, size_t work_bytes, uint8_t* d_out, size_t out_capacity,
+               uint64_t* d_out_bytes, void* stream);
+
+/*
+ * Decode an SHN1 stream (Shannonic §4.2: decTable[X] gives the range s and the bit count; read the
+ * offset o; x = base[s] + o). The stream is self-describing (segments, tables, chunk index);
+ * `p` must equal the parameters it was encoded with (checked on the device) and selects the
+ * kernel configuration. Output: segment after segment, total_symbols bytes.
+ *  d_comp      device, comp_bytes of stream, 16-byte aligned.
+ *  d_work      device workspace of >= shn_decode_workspace_bytes(p) bytes, 256-byte aligned.
+ *  d_out       device, out_capacity bytes, any alignment.
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_UNSUPPORTED (log2L > 8 in this build),
+ *         SHN_ERR_CUDA; device: SHN_ERR_CORRUPT (bad header/descriptor/index, missing sentinel,
+ *         end-of-chunk state or position check failed), SHN_ERR_CAPACITY (out_capacity too small).
+ * A chunk that fails its checks leaves its output bytes unspecified; every other chunk is decoded.
+ */
+int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, void* d_work, size_t work_bytes,
+               uint8_t* d_out, size_t out_capacity, void* stream);
+
+/*
+ * Copy the device status word of a workspace to the host. This call synchronises `stream`
+ * (cudaStreamSynchronize) — it is the one synchronising entry point. h_detail (optional)
+ * receives a hint: the global chunk index of the first failing chunk, or 0.
+ */
+int shn_get_device_status(const void* d_work, uint32_t* h_status, uint32_t* h_detail, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHN_H */
