@@ -29,7 +29,7 @@ TABLE_PUBLIC_BYTES = 800
 EXPORTED = [
     "shn_version", "shn_status_string", "shn_check_params", "shn_table_bytes", "shn_encode_bound",
     "shn_encode_workspace_bytes", "shn_decode_workspace_bytes", "shn_histogram", "shn_build_tables",
-    "shn_encode", "shn_decode", "shn_get_device_status",
+    "shn_encode", "shn_decode", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
 ]
 
 
@@ -84,6 +84,8 @@ def lib():
             "shn_encode": (i32, [vp, vp, u32, vp, P, vp, sz, vp, sz, vp, vp]),
             "shn_decode": (i32, [vp, sz, P, vp, sz, vp, sz, vp]),
             "shn_get_device_status": (i32, [vp, ctypes.POINTER(u32), ctypes.POINTER(u32), vp]),
+            "shn_encode_static_max_chunks": (u64, []),
+            "shn_encode_static": (i32, [vp, vp, u32, vp, P, vp, sz, vp, vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -181,6 +183,20 @@ def shn_encode(x: torch.Tensor, segments, tables: torch.Tensor, p: CodecParams, 
                             len(segments), _dev(tables, "tables") if tables.numel() else None, ctypes.byref(p.c()),
                             _dev(work, "work"), work.numel(), _dev(out, "out"), out.numel(),
                             _dev(out_bytes, "out_bytes"), _stream(stream)), "shn_encode")
+
+
+def shn_encode_static(x: torch.Tensor, segments, tables: torch.Tensor, p: CodecParams, out: torch.Tensor,
+                      out_bytes: torch.Tensor, status: torch.Tensor, stream=None):
+    """shn_encode with the library's built-in scratch array instead of a caller workspace."""
+    xb = _bytes_view(x)
+    _check(lib().shn_encode_static(_dev(xb, "x") if xb.numel() else None, _segments(segments), len(segments),
+                                   _dev(tables, "tables") if tables.numel() else None, ctypes.byref(p.c()),
+                                   _dev(out, "out"), out.numel(), _dev(out_bytes, "out_bytes"),
+                                   _dev(status, "status"), _stream(stream)), "shn_encode_static")
+
+
+def encode_static_max_chunks() -> int:
+    return int(lib().shn_encode_static_max_chunks())
 
 
 def shn_decode(comp: torch.Tensor, comp_bytes: int, p: CodecParams, work: torch.Tensor, out: torch.Tensor,

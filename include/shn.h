@@ -164,6 +164,37 @@ int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, vo
                uint8_t* d_out, size_t out_capacity, void* stream);
 
 /*
+ * shn_encode without a workspace, for callers that cannot allocate device memory. (This entry
+ * point is an addition of this library; the paper has no counterpart.)
+ *
+ * Who needs it: code that must not call cudaMalloc — an allocator or out-of-memory handler, a
+ * plugin whose host application owns all device memory, a path that cannot afford an allocation's
+ * implicit synchronisation. shn_encode needs scratch beyond its inputs and outputs (per-chunk word
+ * counts and their prefix sums); here that scratch is a fixed array inside libshn's own device
+ * memory, sized for SHN_STATIC_MAX_CHUNKS chunks (about 6.3 MB). Every GPU that loads the library
+ * holds this array until the process exits.
+ *
+ *  Arguments are those of shn_encode without d_work/work_bytes, plus
+ *  d_status  device, 8 bytes, 8-byte aligned: receives the device status (as the first 8 bytes of
+ *            shn_encode's workspace would); zeroed by this call.
+ * The stream produced is byte-identical to shn_encode's.
+ * Limits and caveats:
+ *  - more than SHN_STATIC_MAX_CHUNKS chunks in total returns SHN_ERR_CAPACITY (nothing enqueued);
+ *  - the first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *    that device current; make that first call before any stream capture on that device;
+ *  - all calls share the one array: calls whose GPU work overlaps (different streams, or different
+ *    host threads, without ordering between them) race and may produce corrupt streams. Order
+ *    them on one stream or with events.
+ * Never allocates: no cudaMalloc, cudaFree or allocating library routine is called.
+ * Errors: as shn_encode (SHN_ERR_WORKSPACE cannot occur).
+ */
+#define SHN_STATIC_MAX_CHUNKS 524288u
+uint64_t shn_encode_static_max_chunks(void);
+int shn_encode_static(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, const void* d_tables,
+                      const shn_params* p, uint8_t* d_out, size_t out_capacity, uint64_t* d_out_bytes,
+                      uint32_t* d_status, void* stream);
+
+/*
  * Copy the device status word of a workspace to the host. This call synchronises `stream`
  * (cudaStreamSynchronize) — it is the one synchronising entry point. h_detail (optional)
  * receives a hint: the global chunk index of the first failing chunk, or 0.
