@@ -1,22 +1,38 @@
 // decode.cu — chunk-parallel Shannonic/tANS decoder (Shannonic §4.2: "from state X, decTable[X]
 // gives the symbol s and the bit count; read the offset o and restore x = base[s] + o").
 //
-// Layout of the work: a persistent grid of warps; each warp takes 32 consecutive chunks, one per
-// lane. Every lane keeps the decode table of its own chunk's segment in its own shared-memory
-// column ([slot][lane] u32), so all 32 lookups of a warp hit 32 different banks whatever the
-// states are. A table entry packs everything a step needs:
-//   bits 0..4 nb (state bits), 5..8 w (offset bits), 9..16 base' = base ^ 0x80 (output base),
-//   17..28 next slot base.
-// The lane reads its chunk backwards from the end sentinel (FORMAT.md §7) through a 64-bit window
-// refilled one 32-bit word at a time; S interleaved states give independent lookups.
-// Corrupt input never leads to an out-of-bounds access: every offset taken from the stream is
-// checked against the stream and output sizes, the window only ever reads words of the lane's own
-// chunk, and a decoded slot is always < L by construction.
+// Work layout. A persistent grid of 256-thread blocks walks tiles of 256 consecutive chunks; each
+// thread decodes one chunk of C symbols with S interleaved states (FORMAT.md §7), reading the chunk
+// backwards from its end sentinel.
+//
+// Tables. The decode table lives in shared memory as 8-byte entries
+//   .x = shared-memory offset of the next state's row (row base, including this thread's replica)
+//   .y = nb | w << 8 | base' << 16 | (nb + w) << 24      (base' = range base ^ 0x80)
+// so one lookup plus two funnel shifts and one add give the next state's address. When a tile lies
+// in one segment (the common case for large tensors) the table is stored 16 times interleaved
+// ([slot][replica], replica = lane & 15): an 8-byte load is served per half-warp, so the 16 lanes of
+// a half-warp always hit 16 different bank pairs whatever their states — no bank conflicts. Tiles
+// that straddle segments (many small tensors) use plain per-segment copies, built up to 16 at a
+// time. Tables are built in shared memory from the (f, lo) records of the stream.
+//
+// Bits. Each thread keeps a 64-bit window (two words) of its chunk in registers and refills it from
+// a private 128-byte ring in shared memory, which cp.async (16-byte, L2-only) copies fill ahead of
+// use. Two symbols are extracted per window position (fields are <= 16 bits for L <= 256). Decoded
+// bytes go out as 16-byte stores.
+//
+// Robustness. Corrupt input never causes an out-of-bounds access: descriptors and the chunk index
+// are validated against the stream and output sizes, the ring is filled only from the thread's own
+// chunk, and a decoded next-state row is always inside the table by construction.
 #include "shn_internal.cuh"
 
 namespace shn {
 
-constexpr int kDecMaxR = 8;
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr uint32_t kRingQuads = 8;                // 16-byte quads per thread
+constexpr uint32_t kRingBytes = kRingQuads * 16;  // per thread
+constexpr uint32_t kReplicas = 16;
+constexpr uint32_t kStageBytes = 8192;
 
 struct DecHeader {
   uint32_t n_segs, K, R, S, C, tb;
@@ -45,238 +61,410 @@ __device__ __forceinline__ DecHeader read_header(const uint8_t* c) {
   return h;
 }
 
-// One thread validates the header and every segment descriptor / table record (FORMAT.md §6).
-__global__ void decode_check_kernel(const uint8_t* __restrict__ comp, uint64_t comp_bytes, shn_params p,
-                                    DeviceStatus* st, uint64_t out_capacity) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  if (comp_bytes < kHeaderBytes || ld32(comp) != kMagic || (ld32(comp + 4) & 0xFFFFu) != 1u ||
-      (ld32(comp + 4) >> 16) != kHeaderBytes) {
-    report(st, SHN_ERR_CORRUPT, 0);
-    return;
-  }
-  const DecHeader h = read_header(comp);
-  bool ok = h.K == p.K && h.R == p.log2L && h.S == p.states_per_chunk && h.C == p.chunk_symbols &&
-            h.tb == table_record_bytes(h.K) && h.n_segs <= (1u << 30) && h.total_chunks < (1ull << 32);
-  ok = ok && h.index_off == index_offset(h.n_segs, h.K) &&
-       h.payload_off == payload_offset(h.n_segs, h.K, h.total_chunks) && h.stream_bytes <= comp_bytes &&
-       h.payload_off <= h.stream_bytes;
-  if (!ok) {
-    report(st, SHN_ERR_CORRUPT, 0);
-    return;
-  }
-  uint64_t out_off = 0, pay = 0, chunk = 0;
-  for (uint32_t s = 0; s < h.n_segs; ++s) {
-    const uint8_t* d = comp + kHeaderBytes + (uint64_t)kSegDescBytes * s;
-    const uint64_t n = ld64(d);
-    if (n >= (1ull << 32) || ld64(d + 8) != out_off || ld64(d + 16) != pay || ld32(d + 28) != chunk) {
-      report(st, SHN_ERR_CORRUPT, 0);
-      return;
+__device__ __forceinline__ uint32_t width_bits(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
+
+// Validates the header, then every segment descriptor and table record in parallel (each against its
+// successor), so later kernels may trust all offsets taken from them (FORMAT.md §6).
+__global__ void __launch_bounds__(256) decode_check_kernel(const uint8_t* __restrict__ comp, uint64_t comp_bytes,
+                                                           shn_params p, DeviceStatus* st, uint64_t out_capacity) {
+  __shared__ int s_ok;
+  if (threadIdx.x == 0) {
+    int ok = comp_bytes >= kHeaderBytes && ld32(comp) == kMagic && (ld32(comp + 4) & 0xFFFFu) == 1u &&
+             (ld32(comp + 4) >> 16) == kHeaderBytes;
+    if (ok) {
+      const DecHeader h = read_header(comp);
+      ok = h.K == p.K && h.R == p.log2L && h.S == p.states_per_chunk && h.C == p.chunk_symbols &&
+           h.tb == table_record_bytes(h.K) && h.n_segs <= (1u << 30) && h.total_chunks < (1ull << 32) &&
+           h.index_off == index_offset(h.n_segs, h.K) && h.payload_off == payload_offset(h.n_segs, h.K, h.total_chunks) &&
+           h.stream_bytes <= comp_bytes && h.payload_off <= h.stream_bytes && (h.stream_bytes & 15) == 0 &&
+           h.stream_bytes < (1ull << 35);
+      if (ok && h.n_segs == 0) ok = h.total_chunks == 0 && h.total_symbols == 0 && h.stream_bytes == h.payload_off;
     }
-    const uint8_t* rec = comp + kHeaderBytes + (uint64_t)kSegDescBytes * h.n_segs + (uint64_t)h.tb * s;
-    uint32_t fsum = 0, prev_lo = 0;
+    s_ok = ok;
+    if (!ok) report(st, SHN_ERR_CORRUPT, 0);
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const DecHeader h = read_header(comp);
+  const uint8_t* descs = comp + kHeaderBytes;
+  const uint8_t* recs = descs + (uint64_t)kSegDescBytes * h.n_segs;
+  const uint64_t payload_total = h.stream_bytes - h.payload_off;  // includes the final zero padding
+  for (uint32_t s = threadIdx.x; s < h.n_segs; s += blockDim.x) {
+    const uint8_t* d = descs + (uint64_t)kSegDescBytes * s;
+    const uint64_t n = ld64(d), oo = ld64(d + 8), ps = ld64(d + 16);
+    const uint32_t pw = ld32(d + 24), fc = ld32(d + 28);
+    bool ok = n < (1ull << 32) && (ps & 3) == 0;
+    if (s == 0) ok = ok && oo == 0 && ps == 0 && fc == 0;
+    uint64_t n_oo, n_ps, n_fc;
+    if (s + 1 < h.n_segs) {
+      const uint8_t* dn = d + kSegDescBytes;
+      n_oo = ld64(dn + 8);
+      n_ps = ld64(dn + 16);
+      n_fc = ld32(dn + 28);
+      ok = ok && n_ps == ps + 4ull * pw;
+    } else {
+      n_oo = h.total_symbols;
+      n_ps = ps + 4ull * pw;
+      n_fc = h.total_chunks;
+      ok = ok && round_up(h.payload_off + n_ps, 16) == h.stream_bytes;
+    }
+    ok = ok && n_oo == oo + n && n_fc == fc + n_chunks(n, h.C) && ps + 4ull * pw <= payload_total;
+    const uint8_t* rec = recs + (uint64_t)h.tb * s;
+    uint32_t fsum = 0, prev = 0;
     for (uint32_t k = 0; k < h.K; ++k) {
       fsum += (uint32_t)rec[2 * k] | ((uint32_t)rec[2 * k + 1] << 8);
       const uint32_t lo = rec[2 * h.K + k];
-      if ((k == 0 && lo != 0) || (k > 0 && lo <= prev_lo)) ok = false;
-      prev_lo = lo;
+      if ((k == 0 && lo != 0) || (k > 0 && lo <= prev)) ok = false;
+      prev = lo;
     }
-    if (!ok || fsum != (1u << h.R)) {
-      report(st, SHN_ERR_CORRUPT, 0);
-      return;
-    }
-    out_off += n;
-    pay += 4ull * ld32(d + 24);
-    chunk += n_chunks(n, h.C);
+    ok = ok && fsum == (1u << h.R);
+    if (!ok) report(st, SHN_ERR_CORRUPT, 0);
   }
-  if (chunk != h.total_chunks || out_off != h.total_symbols || h.stream_bytes != round_up(h.payload_off + pay, 16)) {
-    report(st, SHN_ERR_CORRUPT, 0);
-    return;
-  }
-  if (h.total_symbols > out_capacity) report(st, SHN_ERR_CAPACITY, 0);
+  if (threadIdx.x == 0 && h.total_symbols > out_capacity) report(st, SHN_ERR_CAPACITY, 0);
 }
 
-// Backward bit reader over the words of one chunk (FORMAT.md §7 "read n bits").
-struct BackReader {
-  const uint32_t* w;
-  unsigned long long buf;  // words k (low) and k+1 (high)
-  int k;
-  int P;                   // unread bits are positions [0, P) of the chunk
-  bool bad;
-  __device__ __forceinline__ void init(const uint32_t* words, int nw) {
-    w = words;
-    const uint32_t last = words[nw - 1];
-    bad = (last == 0u);
-    P = 32 * (nw - 1) + (31 - __clz(last | (bad ? 1u : 0u)));
-    k = P >= 32 ? (P >> 5) - 1 : 0;
-    const uint32_t hi = (k + 1 < nw) ? words[k + 1] : 0u;
-    buf = ((unsigned long long)hi << 32) | words[k];
+// ---- shared-memory decode tables -------------------------------------------------------------
+
+struct SmemLayout {
+  uint32_t table_bytes;  // replicated table (or several plain tables)
+  uint32_t ring_off;
+  uint32_t stage_off;
+  uint32_t stage_per_table;
+  uint32_t max_plain_tables;
+  uint32_t total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
+  SmemLayout l;
+  const uint32_t L = 1u << R;
+  l.table_bytes = L * kReplicas * 8;
+  l.ring_off = l.table_bytes;
+  l.stage_off = l.ring_off + kDecThreads * kRingBytes;
+  l.stage_per_table = (uint32_t)round_up(2 * (K + 1) + 2 * K + 4 * K, 16);
+  uint32_t by_table = l.table_bytes / (L * 8);
+  uint32_t by_stage = kStageBytes / l.stage_per_table;
+  l.max_plain_tables = by_table < by_stage ? by_table : by_stage;
+  if (l.max_plain_tables < 1) l.max_plain_tables = 1;
+  l.total = l.stage_off + kStageBytes;
+  return l;
+}
+
+// Build decode tables (FORMAT.md §5) for segments seg0 .. seg0+nt-1. replicated: nt == 1, entry of
+// slot i, replica c at byte (i*16 + c)*8; plain: table t at t*L*8, entry i at +i*8. All threads of
+// the block take part; the caller synchronises before (readers of the old tables are done).
+__device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, const SmemLayout& lay, uint32_t seg0,
+                                    uint32_t nt, bool replicated, unsigned char* dsm) {
+  const uint32_t K = h.K, R = h.R, L = 1u << R;
+  const uint32_t tid = threadIdx.x;
+  for (uint32_t e = tid; e < nt * K; e += blockDim.x) {
+    const uint32_t t = e / K, k = e - t * K;
+    const uint8_t* rec = recs + (uint64_t)h.tb * (seg0 + t);
+    unsigned char* sg = dsm + lay.stage_off + t * lay.stage_per_table;
+    uint16_t* f = reinterpret_cast<uint16_t*>(sg + 2 * (K + 1));
+    uint32_t* wb = reinterpret_cast<uint32_t*>(sg + 2 * (K + 1) + 2 * K + ((2 * (K + 1) + 2 * K) & 2));
+    const uint32_t lo = rec[2 * K + k];
+    const uint32_t hi = (k + 1 < K) ? rec[2 * K + k + 1] : 256u;
+    f[k] = (uint16_t)((uint32_t)rec[2 * k] | ((uint32_t)rec[2 * k + 1] << 8));
+    wb[k] = width_bits(hi - lo) | (((lo ^ 0x80u) & 0xFFu) << 8);
   }
-  // Read n <= 20 bits ending at P; refill afterwards so that 32 bits stay available.
-  __device__ __forceinline__ uint32_t read(uint32_t n) {
-    int sh = P - (int)n - 32 * k;
-    if (sh < 0) {
-      bad = true;
-      sh = 0;
+  __syncthreads();
+  for (uint32_t t = tid; t < nt; t += blockDim.x) {
+    unsigned char* sg = dsm + lay.stage_off + t * lay.stage_per_table;
+    uint16_t* cumul = reinterpret_cast<uint16_t*>(sg);
+    const uint16_t* f = reinterpret_cast<const uint16_t*>(sg + 2 * (K + 1));
+    uint32_t acc = 0;
+    for (uint32_t k = 0; k < K; ++k) {
+      cumul[k] = (uint16_t)acc;
+      acc += f[k];
     }
-    const uint32_t v = (uint32_t)(buf >> sh) & ((1u << n) - 1u);
-    P -= (int)n;
-    if (P - 32 * k < 32 && k > 0) {
-      --k;
-      buf = (buf << 32) | w[k];
+    cumul[K] = (uint16_t)acc;
+  }
+  __syncthreads();
+  const uint32_t step = (L >> 1) + (L >> 3) + 3;
+  uint32_t inv = step;  // inverse of the odd step modulo 2^32 (Newton), reduced mod L below
+#pragma unroll
+  for (int it = 0; it < 5; ++it) inv *= 2u - step * inv;
+  for (uint32_t e = tid; e < nt * L; e += blockDim.x) {
+    const uint32_t t = e >> R, i = e & (L - 1);
+    const unsigned char* sg = dsm + lay.stage_off + t * lay.stage_per_table;
+    const uint16_t* cumul = reinterpret_cast<const uint16_t*>(sg);
+    const uint16_t* f = reinterpret_cast<const uint16_t*>(sg + 2 * (K + 1));
+    const uint32_t* wb = reinterpret_cast<const uint32_t*>(sg + 2 * (K + 1) + 2 * K + ((2 * (K + 1) + 2 * K) & 2));
+    const uint32_t tau = (i * inv) & (L - 1);  // placement index of slot i
+    int a = 0, b = (int)K - 1;                // its range: largest k with cumul[k] <= tau
+    while (a < b) {
+      const int m = (a + b + 1) >> 1;
+      if (cumul[m] <= tau) a = m;
+      else b = m - 1;
     }
-    return v;
+    const uint32_t s = (uint32_t)a, fs = f[s], c0 = cumul[s];
+    uint32_t rank = 0;  // slots of range s below slot i
+    for (uint32_t u = c0; u < c0 + fs; ++u) rank += (((u * step) & (L - 1)) < i) ? 1u : 0u;
+    const uint32_t x = fs + rank;
+    const uint32_t nb = R - (31u - __clz(x));
+    const uint32_t next = (x << nb) - L;
+    const uint32_t w = wb[s] & 0xFFu, base = wb[s] >> 8;
+    const uint32_t y = nb | (w << 8) | (base << 16) | ((nb + w) << 24);
+    if (replicated) {
+      uint2* row = reinterpret_cast<uint2*>(dsm + i * (kReplicas * 8));
+#pragma unroll
+      for (uint32_t c = 0; c < kReplicas; ++c) row[c] = make_uint2(next * (kReplicas * 8) + c * 8, y);
+    } else {
+      reinterpret_cast<uint2*>(dsm + t * L * 8)[i] = make_uint2(t * L * 8 + next * 8, y);
+    }
+  }
+  __syncthreads();
+}
+
+// ---- per-thread chunk decoder -----------------------------------------------------------------
+
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+struct ChunkCtx {
+  const uint8_t* comp;
+  unsigned char* dsm;
+  uint32_t ring;        // this thread's ring: byte offset in dsm
+  uint32_t ring_saddr;  // ... as a shared-state-space address for cp.async
+  uint64_t cb;          // chunk start, bytes from the stream start
+  uint32_t nw;          // chunk words
+  uint32_t len;         // symbols
+  uint32_t tbase;       // offset of slot 0's entry for this thread (replica / plain table)
+  uint8_t* dst;
+};
+
+// Ring fetcher: quads of 16 bytes (absolute, stream-relative), fetched downwards from the chunk end.
+// (Quad indices fit in 31 bits: streams are limited to 2^35 bytes by the header check.)
+struct Fetcher {
+  int32_t lo;      // lowest quad fetched so far
+  int32_t bottom;  // lowest quad of the chunk
+  __device__ __forceinline__ void fill_to(const ChunkCtx& c, int32_t limit) {
+    const int32_t target = limit > bottom ? limit : bottom;
+    while (lo > target) {
+      --lo;
+      cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
+    }
   }
 };
 
-template <int S>
-__global__ void __launch_bounds__(256) decode_kernel(const uint8_t* __restrict__ comp, DeviceStatus* st,
-                                                     uint8_t* __restrict__ out, uint32_t col_words) {
-  extern __shared__ __align__(16) uint32_t dsm[];
-  if (*(volatile uint32_t*)&st->status != 0) return;
-  const DecHeader h = read_header(comp);
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const uint32_t L = 1u << h.R;
-  // per-warp shared area: table [L][32] u32, spread [L][32] u8, counters [K][32] u8
-  uint32_t* tab = dsm + (size_t)warp * col_words;
-  uint8_t* spread = reinterpret_cast<uint8_t*>(tab + L * 32);
-  uint8_t* cnt = spread + L * 32;
-  const uint32_t step = (L >> 1) + (L >> 3) + 3;
-  const uint8_t* descs = comp + kHeaderBytes;
-  const uint8_t* recs = comp + kHeaderBytes + (uint64_t)kSegDescBytes * h.n_segs;
-  const uint32_t* index = reinterpret_cast<const uint32_t*>(comp + h.index_off);
-  int cur_seg = -1;
-  bool seg_ok = false;
-
-  const uint64_t n_groups = (h.total_chunks + 31) / 32;
-  const uint64_t warps_total = (uint64_t)gridDim.x * (blockDim.x >> 5);
-  for (uint64_t grp = (uint64_t)blockIdx.x * (blockDim.x >> 5) + warp; grp < n_groups; grp += warps_total) {
-    const uint64_t g = grp * 32 + lane;
-    if (g >= h.total_chunks) continue;
-    // segment of chunk g: largest s with first_chunk[s] <= g
-    int a = 0, b = (int)h.n_segs - 1;
-    while (a < b) {
-      const int m = (a + b + 1) >> 1;
-      if (ld32(descs + (uint64_t)kSegDescBytes * m + 28) <= g) a = m;
-      else b = m - 1;
+template <int S, int SH>
+__device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
+  unsigned char* const dsm = c.dsm;
+  const uint32_t mask = kRingBytes - 1;
+  const uint32_t cb_mod = (uint32_t)(c.cb & mask);
+  Fetcher fe;
+  const int32_t q_top = (int32_t)((c.cb + 4ull * c.nw - 1) >> 4);
+  fe.bottom = (int32_t)(c.cb >> 4);
+  fe.lo = q_top + 1;
+  fe.fill_to(c, q_top - (int32_t)kRingQuads + 1);
+  const int32_t cb_words = (int32_t)(c.cb >> 2);  // chunk start in stream words
+  cp_async_commit();
+  cp_async_wait<0>();
+  auto word = [&](int32_t k) -> uint32_t {  // chunk word k (k may be -1: stale, never used validly)
+    return *reinterpret_cast<const uint32_t*>(dsm + c.ring + ((cb_mod + 4u * (uint32_t)k) & mask));
+  };
+  const uint32_t last = word((int32_t)c.nw - 1);
+  if (last == 0u) return false;
+  int32_t P = 32 * ((int32_t)c.nw - 1) + (31 - __clz(last));  // unread bits: [0, P)
+  int32_t thr = P & ~31;                                        // window = words (thr/32 - 1, thr/32)
+  uint32_t rw = (cb_mod + 4u * (uint32_t)((thr >> 5) - 1)) & mask;  // ring offset of word thr/32 - 1
+  uint32_t W1 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + ((rw + 4u) & mask));
+  uint32_t W0 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + rw);
+  auto advance = [&]() {  // keep P in [thr, thr + 32)
+    if (P < thr) {
+      W1 = W0;
+      thr -= 32;
+      rw = (rw - 4u) & mask;
+      W0 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + rw);
     }
-    const int seg = a;
-    const uint8_t* d = descs + (uint64_t)kSegDescBytes * seg;
-    const uint64_t n = ld64(d);
-    const uint64_t out_off = ld64(d + 8);
-    const uint64_t pay_start = ld64(d + 16);
-    const uint32_t pay_words = ld32(d + 24);
-    const uint32_t first = ld32(d + 28);
-    const uint32_t c = (uint32_t)(g - first);
-    const uint32_t nch = (uint32_t)n_chunks(n, h.C);
-    if (c >= nch) continue;  // an empty segment shares its first_chunk with the next one
-    const uint32_t len = (uint32_t)min((uint64_t)h.C, n - (uint64_t)c * h.C);
-
-    if (seg != cur_seg) {
-      cur_seg = seg;
-      // build this lane's decode-table column (FORMAT.md §5)
-      const uint8_t* rec = recs + (uint64_t)h.tb * seg;
-      uint32_t t = 0;
-      for (uint32_t k = 0; k < h.K; ++k) {
-        const uint32_t fk = (uint32_t)rec[2 * k] | ((uint32_t)rec[2 * k + 1] << 8);
-        for (uint32_t r = 0; r < fk && t < L; ++r, ++t) spread[((t * step) & (L - 1)) * 32 + lane] = (uint8_t)k;
-        cnt[k * 32 + lane] = 0;
-      }
-      seg_ok = (t == L);
-      for (uint32_t i = 0; i < L && seg_ok; ++i) {
-        const uint32_t s = spread[i * 32 + lane];
-        const uint32_t j = cnt[s * 32 + lane];
-        cnt[s * 32 + lane] = (uint8_t)(j + 1);
-        const uint32_t fs = (uint32_t)rec[2 * s] | ((uint32_t)rec[2 * s + 1] << 8);
-        const uint32_t x = fs + j;
-        const uint32_t nb = h.R - (31 - __clz(x));
-        const uint32_t nxt = (x << nb) - L;
-        const uint32_t lo = rec[2 * h.K + s];
-        const uint32_t hi = (s + 1 < h.K) ? rec[2 * h.K + s + 1] : 256u;
-        const uint32_t w = (hi - lo <= 1) ? 0u : 32u - __clz(hi - lo - 1);
-        tab[i * 32 + lane] = nb | (w << 5) | ((lo ^ 0x80u) << 9) | (nxt << 17);
-      }
-    }
-    const uint32_t w0 = index[g];
-    const uint32_t w1 = (c + 1 < nch) ? index[g + 1] : pay_words;
-    const uint64_t chunk_byte = h.payload_off + pay_start + 4ull * w0;
-    if (!seg_ok || w1 <= w0 || w1 > pay_words || (c == 0 && w0 != 0) ||
-        h.payload_off + pay_start + 4ull * w1 > h.stream_bytes) {
-      report(st, SHN_ERR_CORRUPT, (uint32_t)g);
-      continue;
-    }
-    BackReader br;
-    br.init(reinterpret_cast<const uint32_t*>(comp + chunk_byte), (int)(w1 - w0));
-    uint32_t X[S];
+  };
+  uint32_t X[S];
 #pragma unroll
-    for (int q = S - 1; q >= 0; --q) X[q] = br.read(h.R);
-    const uint32_t* col = tab + lane;
-    uint8_t* dst = out + out_off + (uint64_t)c * h.C;
-    const bool aligned = ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-    uint32_t i0 = 0;
-    for (; i0 + 16 <= len; i0 += 16) {
-      uint32_t ov[4] = {0u, 0u, 0u, 0u};
+  for (int q = S - 1; q >= 0; --q) {
+    const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
+    X[q] = c.tbase + ((V >> (32u - R)) << SH);
+    P -= (int32_t)R;
+    advance();
+  }
+  const bool aligned = ((reinterpret_cast<uintptr_t>(c.dst) & 15u) == 0);
+  uint32_t i0 = 0;
+  for (; i0 + 16 <= c.len; i0 += 16) {
+    fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    uint32_t ov[4];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        uint32_t& x = X[r & (S - 1)];
-        const uint32_t e = col[x * 32];
-        const uint32_t nb = e & 31u, w = (e >> 5) & 15u;
-        const uint32_t F = br.read(nb + w);
-        x = (e >> 17) + (F >> w);
-        const uint32_t byte = ((e >> 9) + (F & ((1u << w) - 1u))) & 0xFFu;
-        ov[r >> 2] |= byte << (8 * (r & 3));
-      }
-      if (aligned) {
-        *reinterpret_cast<uint4*>(dst + i0) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-      } else {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) dst[i0 + r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
-      }
+    for (int pp = 0; pp < 8; ++pp) {
+      const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
+      const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
+      const uint2 Ea = *reinterpret_cast<const uint2*>(dsm + X[qa]);
+      const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);
+      const uint32_t Va = __funnelshift_l(0u, V, Ea.y);
+      const uint32_t oa = __funnelshift_l(Va, 0u, Ea.y >> 8);
+      const uint32_t ba = oa + (Ea.y >> 16);
+      const uint32_t ta = Ea.y >> 24;
+      X[qa] = Ea.x + (ra << SH);
+      const uint32_t V2 = __funnelshift_l(0u, V, ta);
+      const uint2 Eb = *reinterpret_cast<const uint2*>(dsm + X[qb]);
+      const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
+      const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
+      const uint32_t ob = __funnelshift_l(Vb, 0u, Eb.y >> 8);
+      const uint32_t bb = ob + (Eb.y >> 16);
+      const uint32_t tb = Eb.y >> 24;
+      X[qb] = Eb.x + (rb << SH);
+      P -= (int32_t)(ta + tb);
+      advance();
+      const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
+      if ((pp & 1) == 0) ov[pp >> 1] = pair;
+      else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
     }
-    for (uint32_t i = i0; i < len; ++i) {
-      const int q = (int)(i & (S - 1));
+    if (aligned) {
+      *reinterpret_cast<uint4*>(c.dst + i0) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) c.dst[i0 + r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
+    }
+  }
+  if (i0 < c.len) {
+    fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    cp_async_commit();
+    cp_async_wait<0>();
+    for (uint32_t i = i0; i < c.len; ++i) {
+      const int q = (int)(i % S);
       uint32_t x = X[0];
 #pragma unroll
       for (int k = 1; k < S; ++k)
         if (k == q) x = X[k];
-      const uint32_t e = col[x * 32];
-      const uint32_t nb = e & 31u, w = (e >> 5) & 15u;
-      const uint32_t F = br.read(nb + w);
-      x = (e >> 17) + (F >> w);
-      dst[i] = (uint8_t)(((e >> 9) + (F & ((1u << w) - 1u))) & 0xFFu);
+      const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
+      const uint2 E = *reinterpret_cast<const uint2*>(dsm + x);
+      const uint32_t r = __funnelshift_l(V, 0u, E.y);
+      const uint32_t Vs = __funnelshift_l(0u, V, E.y);
+      const uint32_t o = __funnelshift_l(Vs, 0u, E.y >> 8);
+      x = E.x + (r << SH);
+      P -= (int32_t)(E.y >> 24);
+      advance();
+      c.dst[i] = (uint8_t)(o + (E.y >> 16));
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;
     }
-    bool ok = !br.bad && br.P == 0;
+  }
+  cp_async_wait<0>();
+  bool ok = (P == 0);
 #pragma unroll
-    for (int q = 0; q < S; ++q) ok = ok && (X[q] == 0u);
-    if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+  for (int q = 0; q < S; ++q) ok = ok && (X[q] == c.tbase);
+  return ok;
+}
+
+// ---- the kernel --------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t segment_of(const uint8_t* descs, uint32_t n_segs, uint64_t g) {
+  int a = 0, b = (int)n_segs - 1;  // largest s with first_chunk[s] <= g
+  while (a < b) {
+    const int m = (a + b + 1) >> 1;
+    if (ld32(descs + (uint64_t)kSegDescBytes * m + 28) <= g) a = m;
+    else b = m - 1;
+  }
+  return (uint32_t)a;
+}
+
+template <int S>
+__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const uint8_t* __restrict__ comp, DeviceStatus* st,
+                                                             uint8_t* __restrict__ out) {
+  extern __shared__ __align__(128) unsigned char dsm[];
+  if (*(volatile uint32_t*)&st->status != 0) return;
+  const DecHeader h = read_header(comp);
+  const SmemLayout lay = smem_layout(h.R, h.K);
+  const uint32_t L = 1u << h.R;
+  const uint8_t* descs = comp + kHeaderBytes;
+  const uint8_t* recs = descs + (uint64_t)kSegDescBytes * h.n_segs;
+  const uint32_t* index = reinterpret_cast<const uint32_t*>(comp + h.index_off);
+  const uint32_t tid = threadIdx.x, lane = tid & 31;
+  const uint32_t ring = lay.ring_off + tid * kRingBytes;
+  const uint32_t ring_saddr = (uint32_t)__cvta_generic_to_shared(dsm + ring);
+  const uint64_t n_tiles = (h.total_chunks + kDecThreads - 1) / kDecThreads;
+  int64_t cur_seg = -1;  // segment whose replicated table is in shared memory
+
+  for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const uint64_t g0 = tile * kDecThreads;
+    const uint64_t g_last = min(g0 + kDecThreads, h.total_chunks) - 1;
+    const uint32_t sa = segment_of(descs, h.n_segs, g0), sb = segment_of(descs, h.n_segs, g_last);
+    // this thread's chunk
+    const uint64_t g = g0 + tid;
+    bool valid = g < h.total_chunks;
+    ChunkCtx c;
+    uint32_t seg = 0;
+    if (valid) {
+      seg = segment_of(descs, h.n_segs, g);
+      const uint8_t* d = descs + (uint64_t)kSegDescBytes * seg;
+      const uint64_t n = ld64(d), out_off = ld64(d + 8), pay_start = ld64(d + 16);
+      const uint32_t pay_words = ld32(d + 24), first = ld32(d + 28);
+      const uint32_t ci = (uint32_t)(g - first);
+      const uint32_t nch = (uint32_t)n_chunks(n, h.C);
+      const uint32_t w0 = index[g];
+      const uint32_t w1 = (ci + 1 < nch) ? index[g + 1] : pay_words;
+      if (ci >= nch || w1 <= w0 || w1 > pay_words || (ci == 0 && w0 != 0)) {
+        report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+        valid = false;
+      } else {
+        c.comp = comp;
+        c.dsm = dsm;
+        c.ring = ring;
+        c.ring_saddr = ring_saddr;
+        c.cb = h.payload_off + pay_start + 4ull * w0;
+        c.nw = w1 - w0;
+        c.len = (uint32_t)min((uint64_t)h.C, n - (uint64_t)ci * h.C);
+        c.dst = out + out_off + (uint64_t)ci * h.C;
+      }
+    }
+    if (sa == sb) {
+      if (cur_seg != (int64_t)sa) {
+        __syncthreads();
+        build_decode_tables(recs, h, lay, sa, 1, true, dsm);
+        cur_seg = sa;
+      }
+      if (valid) {
+        c.tbase = (lane & (kReplicas - 1)) * 8;
+        if (!decode_chunk<S, 7>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+      }
+    } else {
+      cur_seg = -1;
+      for (uint32_t s0 = sa; s0 <= sb; s0 += lay.max_plain_tables) {
+        const uint32_t nt = min(lay.max_plain_tables, sb - s0 + 1);
+        __syncthreads();
+        build_decode_tables(recs, h, lay, s0, nt, false, dsm);
+        if (valid && seg >= s0 && seg < s0 + nt) {
+          c.tbase = (seg - s0) * L * 8;
+          if (!decode_chunk<S, 3>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+        }
+      }
+    }
   }
 }
 
 template <int S>
 static cudaError_t launch_decode_t(const uint8_t* d_comp, DeviceStatus* st, uint8_t* d_out, const shn_params& p,
                                    int sm_count, cudaStream_t s) {
-  const uint32_t L = 1u << p.log2L;
-  const uint32_t col_bytes = L * 32 * 4 + L * 32 + p.K * 32;
-  const uint32_t col_words = (col_bytes + 15) / 16 * 4;
-  int warps = (int)((96 * 1024) / (col_words * 4));
-  warps = warps < 1 ? 1 : (warps > 8 ? 8 : warps);
-  const size_t smem = (size_t)warps * col_words * 4;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const SmemLayout lay = smem_layout(p.log2L, p.K);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<S>, warps * 32, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<S>, kDecThreads, lay.total);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  decode_kernel<S><<<sm_count * per_sm, warps * 32, smem, s>>>(d_comp, st, d_out, col_words);
+  decode_kernel<S><<<sm_count * per_sm, kDecThreads, lay.total, s>>>(d_comp, st, d_out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
                           uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s) {
-  decode_check_kernel<<<1, 32, 0, s>>>(d_comp, comp_bytes, p, st, out_capacity);
+  decode_check_kernel<<<1, 256, 0, s>>>(d_comp, comp_bytes, p, st, out_capacity);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (p.states_per_chunk) {
