@@ -87,14 +87,8 @@ size_t shn_table_bytes(const shn_params* p) { return params_ok(p) ? (size_t)SHN_
 size_t shn_encode_bound(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs) {
   uint64_t tc = 0;
   if (!params_ok(p) || !segs_ok(h_segs, n_segs, &tc, nullptr, p->chunk_symbols)) return 0;
-  uint64_t words = 0;
-  for (uint32_t s = 0; s < n_segs; ++s) {
-    const uint64_t nc = n_chunks(h_segs[s].length, p->chunk_symbols);
-    if (nc == 0) continue;
-    const uint64_t last = h_segs[s].length - (nc - 1) * p->chunk_symbols;
-    words += (nc - 1) * chunk_max_words(p->states_per_chunk, p->log2L, p->chunk_symbols) +
-             chunk_max_words(p->states_per_chunk, p->log2L, last);
-  }
+  // every chunk holds at most C symbols (FORMAT.md §6)
+  const uint64_t words = tc * chunk_max_words(p->states_per_chunk, p->log2L, p->chunk_symbols);
   return (size_t)round_up(payload_offset(n_segs, p->K, tc) + 4 * words, 16);
 }
 

@@ -234,9 +234,11 @@ struct ChunkCtx {
   uint32_t ring_saddr;  // ... as a shared-state-space address for cp.async
   uint64_t cb;          // chunk start, bytes from the stream start
   uint32_t nw;          // chunk words
-  uint32_t len;         // symbols
   uint32_t tbase;       // offset of slot 0's entry for this thread (replica / plain table)
-  uint8_t* dst;
+  uint8_t* dst;         // where the chunk's first piece goes (FORMAT.md §6)
+  uint32_t dst_stride;  // bytes between consecutive pieces of the chunk (16 * chunks in its group)
+  uint32_t pieces;
+  uint32_t last_len;    // symbols in the last piece (1..16)
 };
 
 // Ring fetcher: quads of 16 bytes (absolute, stream-relative), fetched downwards from the chunk end.
@@ -293,8 +295,9 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
     advance();
   }
   const bool aligned = ((reinterpret_cast<uintptr_t>(c.dst) & 15u) == 0);
-  uint32_t i0 = 0;
-  for (; i0 + 16 <= c.len; i0 += 16) {
+  const uint32_t full = c.pieces - (c.last_len < 16 ? 1u : 0u);
+  uint8_t* dst = c.dst;
+  for (uint32_t k = 0; k < full; ++k, dst += c.dst_stride) {
     fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<1>();
@@ -325,18 +328,18 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
     }
     if (aligned) {
-      *reinterpret_cast<uint4*>(c.dst + i0) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
     } else {
 #pragma unroll
-      for (int r = 0; r < 16; ++r) c.dst[i0 + r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
+      for (int r = 0; r < 16; ++r) dst[r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
     }
   }
-  if (i0 < c.len) {
+  if (full < c.pieces) {  // the group's short last piece
     fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<0>();
-    for (uint32_t i = i0; i < c.len; ++i) {
-      const int q = (int)(i % S);
+    for (uint32_t i = 0; i < c.last_len; ++i) {
+      const int q = (int)(i % S);  // chunk index 16*full + i, and S divides 16
       uint32_t x = X[0];
 #pragma unroll
       for (int k = 1; k < S; ++k)
@@ -349,7 +352,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       x = E.x + (r << SH);
       P -= (int32_t)(E.y >> 24);
       advance();
-      c.dst[i] = (uint8_t)(o + (E.y >> 16));
+      dst[i] = (uint8_t)(o + (E.y >> 16));
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;
@@ -419,8 +422,11 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const uint8_t* _
         c.ring_saddr = ring_saddr;
         c.cb = h.payload_off + pay_start + 4ull * w0;
         c.nw = w1 - w0;
-        c.len = (uint32_t)min((uint64_t)h.C, n - (uint64_t)ci * h.C);
-        c.dst = out + out_off + (uint64_t)ci * h.C;
+        const ChunkGeo geo = chunk_geo(n, h.C, ci);
+        c.dst = out + out_off + geo.base + 16u * geo.j;
+        c.dst_stride = 16u * geo.m;
+        c.pieces = geo.pieces;
+        c.last_len = geo.last_len;
       }
     }
     if (sa == sb) {

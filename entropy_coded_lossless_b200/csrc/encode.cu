@@ -73,51 +73,58 @@ __device__ __forceinline__ uint32_t enc_step(const EncSmem& sm, uint32_t b, uint
   return o | (r << w);
 }
 
+// Encode one chunk backwards (FORMAT.md §7). seg points at the segment's first byte; the chunk's
+// symbols are its pieces in order (FORMAT.md §6), so the last piece is coded first. Full pieces are
+// read as 16-byte loads, which a warp's 32 chunks of one group issue as 512 consecutive bytes.
 template <int S, bool WRITE>
-__device__ __forceinline__ void encode_chunk(const EncSmem& sm, const uint8_t* src, uint32_t len, uint32_t L,
+__device__ __forceinline__ void encode_chunk(const EncSmem& sm, const uint8_t* seg, const ChunkGeo& g, uint32_t L,
                                              uint32_t R, uint64_t& bits_out, uint32_t& flags, WordWriter* ww) {
   uint32_t X[S];
 #pragma unroll
   for (int q = 0; q < S; ++q) X[q] = L;
   uint64_t bits = 0;
-  const uint32_t tail = len & 15u;
-  // trailing symbols that do not fill a group of 16 (only the last chunk of a segment)
-  for (int i = (int)len - 1; i >= (int)(len - tail); --i) {
-    const int q = i & (S - 1);
-    uint32_t Xq = X[0];
+  int k = (int)g.pieces - 1;
+  if (g.last_len < 16) {  // the group's short last piece, symbol by symbol
+    const uint8_t* src = seg + g.base + 16u * (g.j + (uint32_t)k * g.m);
+    for (int t = (int)g.last_len - 1; t >= 0; --t) {
+      const int q = t & (S - 1);  // chunk index 16k + t, and S divides 16
+      uint32_t Xq = X[0];
 #pragma unroll
-    for (int k = 1; k < S; ++k)
-      if (k == q) Xq = X[k];
-    uint32_t t;
-    const uint32_t field = enc_step(sm, src[i], Xq, t, flags);
+      for (int z = 1; z < S; ++z)
+        if (z == q) Xq = X[z];
+      uint32_t w;
+      const uint32_t field = enc_step(sm, src[t], Xq, w, flags);
 #pragma unroll
-    for (int k = 0; k < S; ++k)
-      if (k == q) X[k] = Xq;
-    bits += t;
-    if (WRITE) ww->put(field, t);
+      for (int z = 0; z < S; ++z)
+        if (z == q) X[z] = Xq;
+      bits += w;
+      if (WRITE) ww->put(field, w);
+    }
+    --k;
   }
-  const bool aligned = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0);
-  for (int i0 = (int)(len - tail) - 16; i0 >= 0; i0 -= 16) {
+  const bool aligned = ((reinterpret_cast<uintptr_t>(seg + g.base) & 15u) == 0);
+  for (; k >= 0; --k) {
+    const uint8_t* src = seg + g.base + 16u * (g.j + (uint32_t)k * g.m);
     uint32_t wv[4];
     if (aligned) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src + i0));
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
       wv[0] = v.x;
       wv[1] = v.y;
       wv[2] = v.z;
       wv[3] = v.w;
     } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        wv[k] = (uint32_t)src[i0 + 4 * k] | ((uint32_t)src[i0 + 4 * k + 1] << 8) |
-                ((uint32_t)src[i0 + 4 * k + 2] << 16) | ((uint32_t)src[i0 + 4 * k + 3] << 24);
+      for (int z = 0; z < 4; ++z)
+        wv[z] = (uint32_t)src[4 * z] | ((uint32_t)src[4 * z + 1] << 8) | ((uint32_t)src[4 * z + 2] << 16) |
+                ((uint32_t)src[4 * z + 3] << 24);
     }
 #pragma unroll
     for (int r = 15; r >= 0; --r) {
       const uint32_t b = (wv[r >> 2] >> (8 * (r & 3))) & 0xFFu;
-      uint32_t t;
-      const uint32_t field = enc_step(sm, b, X[r & (S - 1)], t, flags);
-      bits += t;
-      if (WRITE) ww->put(field, t);
+      uint32_t w;
+      const uint32_t field = enc_step(sm, b, X[r & (S - 1)], w, flags);
+      bits += w;
+      if (WRITE) ww->put(field, w);
     }
   }
 #pragma unroll
@@ -142,10 +149,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t
   const uint32_t len_seg = b.length[seg];
   const uint32_t nch = (uint32_t)n_chunks(len_seg, lay.C);
   if (c >= nch) return;
-  const uint32_t len = min(lay.C, len_seg - c * lay.C);
+  const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   uint64_t bits = 0;
   uint32_t flags = 0;
-  encode_chunk<S, false>(sm, in + b.offset[seg] + (uint64_t)c * lay.C, len, L, lay.R, bits, flags, nullptr);
+  encode_chunk<S, false>(sm, in + b.offset[seg], geo, L, lay.R, bits, flags, nullptr);
   const uint64_t total = bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
   if ((flags & 0x80000000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
@@ -168,7 +175,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   const uint32_t len_seg = b.length[seg];
   const uint32_t nch = (uint32_t)n_chunks(len_seg, lay.C);
   if (c >= nch) return;
-  const uint32_t len = min(lay.C, len_seg - c * lay.C);
+  const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
   WordWriter ww;
   ww.out = reinterpret_cast<uint32_t*>(out + lay.payload_offset) + w.word_offset[g];
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   ww.cnt = 0;
   uint64_t bits = 0;
   uint32_t flags = 0;
-  encode_chunk<S, true>(sm, in + b.offset[seg] + (uint64_t)c * lay.C, len, L, lay.R, bits, flags, &ww);
+  encode_chunk<S, true>(sm, in + b.offset[seg], geo, L, lay.R, bits, flags, &ww);
   ww.put(1u, 1u);  // sentinel
   if (ww.cnt > 0 && ww.out < ww.end) *ww.out = (uint32_t)ww.acc;
 }

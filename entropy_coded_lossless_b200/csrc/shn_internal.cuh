@@ -31,6 +31,34 @@ __host__ __device__ inline uint64_t chunk_max_words(uint32_t S, uint32_t R, uint
   return ((uint64_t)S * R + c * (uint64_t)(R + 8) + 1 + 31) / 32;
 }
 
+// ---- which symbols a chunk holds (FORMAT.md §6) -----------------------------------------------
+// Chunks come in groups of up to 32; a group's symbols are cut into 16-symbol pieces dealt round
+// robin to its chunks. Chunk c of a segment of n symbols: group base symbol, index j in the group,
+// stride m (chunks in the group), number of pieces, and the length of its last piece (1..16).
+struct ChunkGeo {
+  uint32_t base;      // first symbol of the group (relative to the segment)
+  uint32_t j;         // chunk index within the group
+  uint32_t m;         // chunks in the group: piece k of this chunk starts at base + 16*(j + k*m)
+  uint32_t pieces;
+  uint32_t last_len;  // symbols in the last piece
+};
+
+__host__ __device__ inline ChunkGeo chunk_geo(uint64_t n, uint32_t C, uint32_t c) {
+  ChunkGeo g;
+  const uint64_t nch = n_chunks(n, C);
+  const uint32_t grp = c >> 5;
+  g.j = c & 31u;
+  g.m = (uint32_t)((nch - 32ull * grp) < 32 ? (nch - 32ull * grp) : 32);
+  const uint64_t base = 32ull * grp * C;
+  const uint64_t end = (32ull * (grp + 1) * C < n) ? 32ull * (grp + 1) * C : n;
+  const uint32_t ng = (uint32_t)(end - base);
+  const uint32_t P = (ng + 15) >> 4;
+  g.base = (uint32_t)base;
+  g.pieces = (P - g.j + g.m - 1) / g.m;
+  g.last_len = (g.j + (g.pieces - 1) * g.m == P - 1) ? ng - 16 * (P - 1) : 16u;
+  return g;
+}
+
 // ---- device table record (include/shn.h: shn_table) -----------------------------------------
 // opaque part: uint2 sym[256] for every raw byte b (u = b ^ 0x80):
 //   .x = bias[s]  (nb = (X + bias) >> 16),

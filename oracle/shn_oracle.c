@@ -387,18 +387,32 @@ static int params_ok(const orc_params* p) {
 
 static uint64_t seg_chunks(uint64_t n, int C) { return (n + (uint64_t)C - 1) / (uint64_t)C; }
 
+/* FORMAT.md §6 "which symbols a chunk holds": chunks come in groups of up to 32; a group's symbols
+ * are cut into 16-symbol pieces dealt round-robin to its chunks. Writes the positions (relative to
+ * the segment start) of chunk c's symbols, in chunk order, to pos (if not NULL); returns the count. */
+static uint32_t chunk_positions(uint64_t n, int C, uint64_t c, uint64_t* pos) {
+  const uint64_t nch = seg_chunks(n, C);
+  const uint64_t grp = c / 32, j = c % 32;
+  const uint64_t m = (nch - 32 * grp < 32) ? nch - 32 * grp : 32;
+  const uint64_t base = 32 * grp * (uint64_t)C;
+  const uint64_t end = (32 * (grp + 1) * (uint64_t)C < n) ? 32 * (grp + 1) * (uint64_t)C : n;
+  const uint64_t ng = end - base;
+  const uint64_t P = (ng + 15) / 16;
+  uint32_t count = 0;
+  for (uint64_t p = j; p < P; p += m)
+    for (uint64_t t = 0; t < 16 && 16 * p + t < ng; t++) {
+      if (pos) pos[count] = base + 16 * p + t;
+      count++;
+    }
+  return count;
+}
+
 uint64_t orc_stream_bound(const orc_params* p, const orc_segment* segs, int n_segs) {
   if (!params_ok(p) || n_segs < 0) return 0;
   uint64_t tb = round_up(3ull * (uint64_t)p->K, 4);
-  uint64_t chunks = 0, words = 0;
-  for (int s = 0; s < n_segs; s++) {
-    uint64_t nc = seg_chunks(segs[s].length, p->C);
-    chunks += nc;
-    for (uint64_t c = 0; c < nc; c++) {
-      uint64_t len = (c + 1 < nc) ? (uint64_t)p->C : segs[s].length - c * (uint64_t)p->C;
-      words += chunk_max_words(p->S, p->R, len);
-    }
-  }
+  uint64_t chunks = 0;
+  for (int s = 0; s < n_segs; s++) chunks += seg_chunks(segs[s].length, p->C);
+  uint64_t words = chunks * chunk_max_words(p->S, p->R, (uint64_t)p->C); /* every chunk holds <= C symbols */
   uint64_t index_off = 64 + 32ull * (uint64_t)n_segs + tb * (uint64_t)n_segs;
   uint64_t payload_off = round_up(index_off + 4 * chunks, 16);
   return round_up(payload_off + 4 * words, 16);
@@ -499,23 +513,29 @@ static void enc_chunk(void* vctx, uint64_t g) {
   uint64_t s = ctx->chunk_seg[g], c = ctx->chunk_local[g];
   const orc_segment* sg = &ctx->segs[s];
   const int C = ctx->p->C;
-  uint64_t nc = seg_chunks(sg->length, C);
-  uint32_t len = (uint32_t)((c + 1 < nc) ? (uint64_t)C : sg->length - c * (uint64_t)C);
   if (ctx->seg_rc[s] != ORC_OK) {
     ctx->chunk_nwords[g] = -ctx->seg_rc[s];
     return;
   }
+  uint64_t* pos = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)C);
+  uint8_t* sym = (uint8_t*)malloc((size_t)C);
+  const uint32_t len = chunk_positions(sg->length, C, c, pos);
   uint64_t cap = chunk_max_words(ctx->p->S, ctx->p->R, len) + 1;
   uint32_t* w = (uint32_t*)malloc(sizeof(uint32_t) * cap);
-  if (!w) {
+  if (!w || !pos || !sym) {
+    free(w);
+    free(pos);
+    free(sym);
     ctx->chunk_nwords[g] = -ORC_ERR_NOMEM;
     return;
   }
+  for (uint32_t i = 0; i < len; i++) sym[i] = ctx->input[sg->offset + pos[i]];
   uint64_t bits = 0;
-  ctx->chunk_nwords[g] = orc_encode_chunk(&ctx->tables[s], ctx->p->S, ctx->input + sg->offset + c * (uint64_t)C,
-                                          len, w, cap, &bits);
+  ctx->chunk_nwords[g] = orc_encode_chunk(&ctx->tables[s], ctx->p->S, sym, len, w, cap, &bits);
   ctx->chunk_words[g] = w;
   ctx->chunk_bits[g] = bits;
+  free(pos);
+  free(sym);
 }
 
 static int encode_stream_impl(const uint8_t* input, const orc_segment* segs, int n_segs, const orc_params* p,
@@ -687,7 +707,6 @@ static void dec_chunk(void* vctx, uint64_t g) {
   uint64_t s = ctx->chunk_seg[g];
   uint64_t c = g - ctx->seg_first_chunk[s];
   uint64_t nc = seg_chunks(ctx->seg_nsym[s], ctx->C);
-  uint32_t len = (uint32_t)((c + 1 < nc) ? (uint64_t)ctx->C : ctx->seg_nsym[s] - c * (uint64_t)ctx->C);
   uint64_t w0 = get32(ctx->stream + ctx->index_off + 4 * g);
   uint64_t w1 = (c + 1 < nc) ? get32(ctx->stream + ctx->index_off + 4 * (g + 1)) : ctx->seg_pay_words[s];
   if (w1 <= w0 || w1 > ctx->seg_pay_words[s] || (c == 0 && w0 != 0)) {
@@ -697,15 +716,23 @@ static void dec_chunk(void* vctx, uint64_t g) {
   /* words are little-endian in the stream; copy them out so the reader works on host ints */
   uint64_t nw = w1 - w0;
   uint32_t* words = (uint32_t*)malloc(sizeof(uint32_t) * nw);
-  if (!words) {
+  uint64_t* pos = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)ctx->C);
+  uint8_t* sym = (uint8_t*)malloc((size_t)ctx->C);
+  if (!words || !pos || !sym) {
+    free(words);
+    free(pos);
+    free(sym);
     ctx->chunk_rc[g] = ORC_ERR_NOMEM;
     return;
   }
+  const uint32_t len = chunk_positions(ctx->seg_nsym[s], ctx->C, c, pos);
   const uint8_t* base = ctx->stream + ctx->payload_off + ctx->seg_pay_start[s] + 4 * w0;
   for (uint64_t k = 0; k < nw; k++) words[k] = get32(base + 4 * k);
-  ctx->chunk_rc[g] = orc_decode_chunk(&ctx->tables[s], ctx->S, words, nw, len,
-                                      ctx->out + ctx->seg_out_off[s] + c * (uint64_t)ctx->C);
+  ctx->chunk_rc[g] = orc_decode_chunk(&ctx->tables[s], ctx->S, words, nw, len, sym);
+  for (uint32_t i = 0; i < len; i++) ctx->out[ctx->seg_out_off[s] + pos[i]] = sym[i];
   free(words);
+  free(pos);
+  free(sym);
 }
 
 int orc_decode_stream(const uint8_t* stream, uint64_t bytes, int n_threads, uint8_t* out, uint64_t cap,

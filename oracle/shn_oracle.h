@@ -77,7 +77,8 @@ int orc_normalize(const uint64_t* N, int K, int R, uint32_t* f);
 int orc_tables_init(const uint16_t* lo, const uint32_t* f, int K, int R, orc_tables* t);
 int orc_build_segment_tables(const uint64_t hist[256], int K, int R, orc_tables* t, int64_t* dp_cost);
 
-/* One chunk. Symbols are u = byte ^ 0x80. Returns words written, or -(error). */
+/* One chunk, given its symbol sequence (FORMAT.md §6 says which tensor positions a chunk holds).
+ * Symbols are u = byte ^ 0x80. Returns words written, or -(error). */
 int64_t orc_encode_chunk(const orc_tables* t, int S, const uint8_t* bytes, uint32_t c, uint32_t* words,
                          uint64_t cap_words, uint64_t* payload_bits);
 int orc_decode_chunk(const orc_tables* t, int S, const uint32_t* words, uint64_t nwords, uint32_t c,

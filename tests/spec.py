@@ -35,6 +35,20 @@ def parse_stream(buf):
                 segments=segs, index=index, raw=b)
 
 
+def chunk_positions(n, C, c):
+    """FORMAT.md §6: positions (relative to the segment start) of chunk c's symbols, in order."""
+    nch = -(-n // C)
+    grp, j = divmod(c, 32)
+    m = min(32, nch - 32 * grp)
+    base = 32 * grp * C
+    ng = min(32 * (grp + 1) * C, n) - base
+    P = -(-ng // 16)
+    out = []
+    for p in range(j, P, m):
+        out.extend(base + 16 * p + t for t in range(16) if 16 * p + t < ng)
+    return out
+
+
 def chunk_words(st, seg_id, c):
     """Words of chunk c of segment seg_id (a numpy uint32 array)."""
     sg = st["segments"][seg_id]

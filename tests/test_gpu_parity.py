@@ -168,8 +168,8 @@ def _sampled_chunk_check(orc, x_dev, segs, p, g_stream, n_samples=24, seed=0):
         sg = st["segments"][si]
         nch = -(-n // p.chunk_symbols)
         c = int(rng.integers(0, nch))
-        clen = min(p.chunk_symbols, n - c * p.chunk_symbols)
-        chunk = x_dev[o + c * p.chunk_symbols: o + c * p.chunk_symbols + clen].cpu().numpy().view(np.uint8)
+        pos = torch.tensor(spec.chunk_positions(n, p.chunk_symbols, c), dtype=torch.int64, device=x_dev.device)
+        chunk = x_dev[o + pos].cpu().numpy().view(np.uint8)
         t = orc.tables(np.array(sg["lo"], np.uint16), np.array(sg["f"], np.uint32), p.log2L)
         words, _ = orc.encode_chunk(t, p.states_per_chunk, chunk)
         assert np.array_equal(spec.chunk_words(st, si, c), words), (si, c)

@@ -255,7 +255,7 @@ def test_k1_payload_is_reversed_raw_bytes(orc):
     u = x.view(np.uint8) ^ 0x80
     for c in range(3):
         words = spec.chunk_words(st, 0, c)
-        seg = u[c * 1024:(c + 1) * 1024]
+        seg = u[spec.chunk_positions(x.size, 1024, c)]
         raw = words.tobytes()
         assert raw[: seg.size] == seg[::-1].tobytes()
         rest = int.from_bytes(raw[seg.size:], "little")
@@ -280,6 +280,23 @@ def test_single_value_has_empty_payload(orc):
     assert stats[0].payload_bits == 0
 
 
+def test_chunk_mapping_partitions_each_segment():
+    """FORMAT.md §6: the chunks of a segment hold every symbol exactly once, at most C each, and in
+    a full group of 32 the k-th pieces of the chunks are 512 consecutive symbols."""
+    for n, C in [(0, 128), (1, 128), (128, 128), (129, 128), (5000, 256), (32 * 256, 256), (33 * 256 + 7, 256),
+                 (70 * 1024 + 3, 1024), (1_000_003, 4096)]:
+        nch = -(-n // C)
+        seen = np.zeros(n, np.int64)
+        for c in range(nch):
+            pos = spec.chunk_positions(n, C, c)
+            assert 0 < len(pos) <= C
+            seen[pos] += 1
+        assert (seen == 1).all()
+        if n >= 32 * C:
+            firsts = [spec.chunk_positions(n, C, c)[16 * 3] for c in range(32)]
+            assert firsts == list(range(firsts[0], firsts[0] + 512, 16))
+
+
 def test_independent_reader_decodes_oracle_stream(orc):
     rng = np.random.default_rng(4)
     for trial in range(4):
@@ -292,10 +309,9 @@ def test_independent_reader_decodes_oracle_stream(orc):
         for si, sg in enumerate(st["segments"]):
             nch = -(-sg["n"] // 256)
             for c in range(nch):
-                clen = min(256, sg["n"] - 256 * c)
-                got, ok = spec.spec_decode_chunk(spec.chunk_words(st, si, c), sg["lo"], sg["f"], R, S, clen)
-                start = sg["out_offset"] + 256 * c
-                assert ok and got == u[start:start + clen].tolist()
+                pos = sg["out_offset"] + np.array(spec.chunk_positions(sg["n"], 256, c), dtype=np.int64)
+                got, ok = spec.spec_decode_chunk(spec.chunk_words(st, si, c), sg["lo"], sg["f"], R, S, pos.size)
+                assert ok and got == u[pos].tolist()
 
 
 def test_corruption_is_reported(orc):
