@@ -149,6 +149,8 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
   if ((reinterpret_cast<uintptr_t>(d_out) & 15) || (reinterpret_cast<uintptr_t>(d_work) & 255) ||
       (reinterpret_cast<uintptr_t>(d_out_bytes) & 7) || (d_tables && (reinterpret_cast<uintptr_t>(d_tables) & 255)))
     return SHN_ERR_INVALID_ARG;
+  // word offsets inside the payload are 32-bit: streams are limited to 16 GiB
+  if (shn_encode_bound(p, h_segs, n_segs) > (16ull << 30)) return SHN_ERR_INVALID_ARG;
   const EncWorkLayout wl = enc_work_layout(tc);
   if (work_bytes < wl.total) return SHN_ERR_WORKSPACE;
   EncodeLayout lay;

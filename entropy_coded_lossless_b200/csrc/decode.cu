@@ -7,8 +7,11 @@
 //
 // Tables. The decode table lives in shared memory as 8-byte entries
 //   .x = shared-memory offset of the next state's row (row base, including this thread's replica)
-//   .y = nb | w << 8 | base' << 16 | (nb + w) << 24      (base' = range base ^ 0x80)
-// so one lookup plus two funnel shifts and one add give the next state's address. When a tile lies
+//   .y = nb | w << 8 | base' << 16 | (-(nb + w) & 0xFF) << 24     (base' = range base ^ 0x80)
+// so one lookup plus two funnel shifts and one multiply-add give the next state's address. The
+// fields above bit 7 are read with multiply-high instructions (y >> s == mulhi(y, 2^(32-s)), and a
+// signed mulhi by 2^8 yields the negated field width), which run on the FMA pipe and leave the ALU
+// pipe to the funnel shifts. When a tile lies
 // in one segment (the common case for large tensors) the table is stored 16 times interleaved
 // ([slot][replica], replica = lane & 15): an 8-byte load is served per half-warp, so the 16 lanes of
 // a half-warp always hit 16 different bank pairs whatever their states — no bank conflicts. Tiles
@@ -204,7 +207,7 @@ __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, con
     const uint32_t nb = R - (31u - __clz(x));
     const uint32_t next = (x << nb) - L;
     const uint32_t w = wb[s] & 0xFFu, base = wb[s] >> 8;
-    const uint32_t y = nb | (w << 8) | (base << 16) | ((nb + w) << 24);
+    const uint32_t y = nb | (w << 8) | (base << 16) | (((0u - (nb + w)) & 0xFFu) << 24);
     if (replicated) {
       uint2* row = reinterpret_cast<uint2*>(dsm + i * (kReplicas * 8));
 #pragma unroll
@@ -225,6 +228,19 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// y >> 8, y >> 16 and the signed top byte, computed on the FMA pipe (see the file comment).
+__device__ __forceinline__ uint32_t shr8_fma(uint32_t y) { return __umulhi(y, 1u << 24); }
+__device__ __forceinline__ uint32_t add_shr16_fma(uint32_t y, uint32_t a) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(y), "r"(1u << 16), "r"(a));
+  return d;
+}
+__device__ __forceinline__ int32_t add_top_byte_fma(uint32_t y, int32_t p) {  // p + (int8)(y >> 24)
+  int32_t d;
+  asm("mad.hi.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(y), "r"(256), "r"(p));
+  return d;
 }
 
 struct ChunkCtx {
@@ -305,23 +321,24 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
 #pragma unroll
     for (int pp = 0; pp < 8; ++pp) {
       const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
-      const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
+      const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);  // next 32 bits, top-aligned
       const uint2 Ea = *reinterpret_cast<const uint2*>(dsm + X[qa]);
-      const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);
-      const uint32_t Va = __funnelshift_l(0u, V, Ea.y);
-      const uint32_t oa = __funnelshift_l(Va, 0u, Ea.y >> 8);
-      const uint32_t ba = oa + (Ea.y >> 16);
-      const uint32_t ta = Ea.y >> 24;
-      X[qa] = Ea.x + (ra << SH);
-      const uint32_t V2 = __funnelshift_l(0u, V, ta);
+      const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);          // state bits: top nb of V
+      const uint32_t Va = __funnelshift_l(0u, V, Ea.y);          // V << nb
+      const uint32_t wa = shr8_fma(Ea.y);                        // low 5 bits: w
+      const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
+      const uint32_t ba = add_shr16_fma(Ea.y, oa);               // low byte: base' + offset
+      X[qa] = Ea.x + ra * (1u << SH);
+      const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
+      P = add_top_byte_fma(Ea.y, P);                             // P -= nb + w
       const uint2 Eb = *reinterpret_cast<const uint2*>(dsm + X[qb]);
       const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
       const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
-      const uint32_t ob = __funnelshift_l(Vb, 0u, Eb.y >> 8);
-      const uint32_t bb = ob + (Eb.y >> 16);
-      const uint32_t tb = Eb.y >> 24;
-      X[qb] = Eb.x + (rb << SH);
-      P -= (int32_t)(ta + tb);
+      const uint32_t wb = shr8_fma(Eb.y);
+      const uint32_t ob = __funnelshift_l(Vb, 0u, wb);
+      const uint32_t bb = add_shr16_fma(Eb.y, ob);
+      X[qb] = Eb.x + rb * (1u << SH);
+      P = add_top_byte_fma(Eb.y, P);
       advance();
       const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
       if ((pp & 1) == 0) ov[pp >> 1] = pair;
@@ -348,11 +365,11 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       const uint2 E = *reinterpret_cast<const uint2*>(dsm + x);
       const uint32_t r = __funnelshift_l(V, 0u, E.y);
       const uint32_t Vs = __funnelshift_l(0u, V, E.y);
-      const uint32_t o = __funnelshift_l(Vs, 0u, E.y >> 8);
-      x = E.x + (r << SH);
-      P -= (int32_t)(E.y >> 24);
+      const uint32_t o = __funnelshift_l(Vs, 0u, shr8_fma(E.y));
+      x = E.x + r * (1u << SH);
+      P = add_top_byte_fma(E.y, P);
       advance();
-      dst[i] = (uint8_t)(o + (E.y >> 16));
+      dst[i] = (uint8_t)add_shr16_fma(E.y, o);
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;

@@ -1,32 +1,38 @@
 // encode.cu — chunk-parallel Shannonic/tANS encoder (Shannonic §4.2, Algorithm 2).
 //
 // Per value x (symbol u = x ^ 0x80): s = rangeId[u]; emit the offset u - base[s] in nb[s] bits;
-// emit the low state bits that renormalise X for s (count = (X + bias[s]) >> 16); move X through
-// encTable[start[s] + (X >> nb)]. Only table lookups, shifts, masks and adds (§4.2: no multiply or
-// divide on the critical path). Chunks of C symbols are independent (FORMAT.md §7): one thread
-// encodes one chunk backwards with S interleaved states.
+// emit the low state bits that renormalise X for s; move X through encTable (§4.2: table lookups,
+// shifts, masks and adds only). Chunks are independent (FORMAT.md §7): one thread encodes one chunk
+// backwards with S interleaved states.
 //
 // The stream position of a chunk depends on the sizes of all chunks before it, so encoding runs
 // in passes: (1) every thread runs its chunk's state machine and records the chunk's word count,
 // (2) an exclusive scan turns counts into word offsets, (3) the header, segment descriptors, table
 // records and chunk index are written, (4) every thread re-runs its chunk and writes the words to
 // their final place. No device-wide spin waits; everything is ordered by the stream.
+//
+// Shared-memory tables. Each block codes chunks of one segment. When the (range, state) product
+// fits, the block expands the segment's table into one step table
+//   T[s][slot] = next slot | nb << 12     (nb = renormalisation bits of state L + slot for range s)
+// and a byte table B[b] = s | w << 8 | offset << 16 | absent << 31, both stored several times
+// interleaved ([entry][replica], replica from the lane index) so that a warp's lookups spread over
+// the banks instead of colliding. Otherwise it keeps Algorithm 2's per-range bias/start form.
 #include "shn_internal.cuh"
 
 namespace shn {
 
 constexpr int kEncThreads = 128;
+constexpr uint32_t kByteReplicas = 4;
+constexpr uint32_t kStepTableBudget = 16384;  // bytes of shared memory for the replicated T
+constexpr uint32_t kRingWords = 32;           // per-thread output staging ring (write pass)
+constexpr uint32_t kRingStride = kRingWords + 4;  // 144-byte rows: 16-byte reads of 8 rows hit distinct banks
 
-struct EncSmem {
-  uint2 sym[256];
-  uint16_t enc[4096];
-};
-
-__device__ __forceinline__ void load_tables(EncSmem& sm, const shn_table* t, uint32_t L) {
-  const uint2* sym = table_sym(t);
-  const uint16_t* enc = table_enc(t);
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.sym[i] = sym[i];
-  for (uint32_t i = threadIdx.x; i < L; i += blockDim.x) sm.enc[i] = enc[i];
+__host__ __device__ inline uint32_t step_replicas(uint32_t K, uint32_t R) {
+  const uint32_t bytes = K * (1u << R) * 2u;
+  if (bytes > kStepTableBudget) return 0;  // step table does not fit: per-range form
+  uint32_t r = 8;
+  while (r > 1 && bytes * r > kStepTableBudget) r >>= 1;
+  return r;
 }
 
 // Segment of this block: largest s with block_start[s] <= blockIdx.x.
@@ -40,67 +46,134 @@ __device__ __forceinline__ int block_segment(const EncBatch& b) {
   return lo;
 }
 
-// Bit sink of the write pass: LSB-first appends, 32-bit words stored as they fill.
-struct WordWriter {
-  uint32_t* out;
-  uint32_t* end;  // first word past this chunk (the size pass counted exactly this many)
-  unsigned long long acc;
-  uint32_t cnt;
-  __device__ __forceinline__ void put(uint32_t v, uint32_t n) {
-    acc |= (unsigned long long)v << cnt;
-    cnt += n;
-    if (cnt >= 32) {
-      if (out < end) *out = (uint32_t)acc;
-      ++out;
-      acc >>= 32;
-      cnt -= 32;
-    }
+// ---- the two table forms ---------------------------------------------------------------------
+
+// Replicated step table form. State is the slot X - L.
+struct StepCoder {
+  const uint32_t* B;   // [256][kByteReplicas]
+  const uint16_t* T;   // [K*L][rep]
+  uint32_t R, rep_shift, brep, trep;
+  __device__ __forceinline__ uint32_t init_state(uint32_t) const { return 0u; }
+  __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st; }  // X - L
+  // one symbol: returns the field (offset low, state bits high), its width, the new state
+  __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& st, uint32_t& width, uint32_t& flags) const {
+    const uint32_t e = B[(b << 2) + brep];
+    const uint32_t sidx = ((e & 0xFFu) << R) | st;
+    const uint32_t tv = T[(sidx << rep_shift) + trep];
+    const uint32_t nb = tv >> 12;
+    const uint32_t w = (e >> 8) & 0xFu;
+    const uint32_t r = st & ~(0xFFFFFFFFu << nb);
+    flags |= e;
+    st = tv & 0xFFFu;
+    width = w + nb;
+    return ((e >> 16) & 0xFFu) | (r << w);
   }
 };
 
-// One encoder step for symbol byte b in state X. Returns the field (offset low, state bits high)
-// and its width; updates X.
-__device__ __forceinline__ uint32_t enc_step(const EncSmem& sm, uint32_t b, uint32_t& X, uint32_t& width,
-                                             uint32_t& flags) {
-  const uint2 e = sm.sym[b];
-  const uint32_t nb = (X + e.x) >> 16;
-  const uint32_t w = (e.y >> 24) & 15u;
-  const uint32_t o = (e.y >> 16) & 0xFFu;
-  const uint32_t r = X & ((1u << nb) - 1u);
-  X = sm.enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)];
-  flags |= e.y;
-  width = w + nb;
-  return o | (r << w);
+// Per-range form (Algorithm 2's bias/start): sym[raw byte] = {bias, (start + 4096) | o << 16 | w << 24}.
+struct RangeCoder {
+  const uint2* sym;
+  const uint16_t* enc;
+  uint32_t L;
+  __device__ __forceinline__ uint32_t init_state(uint32_t) const { return L; }
+  __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st - L; }
+  __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
+    const uint2 e = sym[b];
+    const uint32_t nb = (X + e.x) >> 16;
+    const uint32_t w = (e.y >> 24) & 15u;
+    const uint32_t o = (e.y >> 16) & 0xFFu;
+    const uint32_t r = X & ((1u << nb) - 1u);
+    X = enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)];
+    flags |= e.y;
+    width = w + nb;
+    return o | (r << w);
+  }
+};
+
+__host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t K, uint32_t R) {
+  const uint32_t rep = step_replicas(K, R);
+  if (rep) return 256 * kByteReplicas * 4 + K * (1u << R) * 2 * rep;
+  return 256 * 8 + (1u << R) * 2;
 }
 
-// Encode one chunk backwards (FORMAT.md §7). seg points at the segment's first byte; the chunk's
-// symbols are its pieces in order (FORMAT.md §6), so the last piece is coded first. Full pieces are
-// read as 16-byte loads, which a warp's 32 chunks of one group issue as 512 consecutive bytes.
-template <int S, bool WRITE>
-__device__ __forceinline__ void encode_chunk(const EncSmem& sm, const uint8_t* seg, const ChunkGeo& g, uint32_t L,
-                                             uint32_t R, uint64_t& bits_out, uint32_t& flags, WordWriter* ww) {
-  uint32_t X[S];
+// Expand table record t into shared memory (all threads of the block).
+template <bool STEP>
+__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t K, uint32_t R,
+                                           StepCoder& sc, RangeCoder& rc) {
+  const uint32_t L = 1u << R;
+  const uint2* sym = table_sym(t);
+  const uint16_t* enc = table_enc(t);
+  const uint32_t lane = threadIdx.x & 31;
+  if (STEP) {
+    const uint32_t rep = step_replicas(K, R);
+    uint32_t* B = reinterpret_cast<uint32_t*>(smem);
+    uint16_t* T = reinterpret_cast<uint16_t*>(smem + 256 * kByteReplicas * 4);
+    for (uint32_t b = threadIdx.x; b < 256; b += blockDim.x) {
+      const uint32_t u = b ^ 0x80u;
+      int lo = 0, hi = (int)K - 1;  // range of u: largest k with lo[k] <= u
+      while (lo < hi) {
+        const int m = (lo + hi + 1) >> 1;
+        if (t->lo[m] <= u) lo = m;
+        else hi = m - 1;
+      }
+      const uint32_t e = sym[b].y;  // offset and width as the record stores them
+      const uint32_t v = (uint32_t)lo | (((e >> 24) & 15u) << 8) | (((e >> 16) & 0xFFu) << 16) | (e & 0x80000000u);
 #pragma unroll
-  for (int q = 0; q < S; ++q) X[q] = L;
-  uint64_t bits = 0;
+      for (uint32_t c = 0; c < kByteReplicas; ++c) B[b * kByteReplicas + c] = v;
+    }
+    for (uint32_t i = threadIdx.x; i < K * L; i += blockDim.x) {
+      const uint32_t s = i >> R, slot = i & (L - 1);
+      uint32_t v = 0;
+      if (t->f[s] != 0) {
+        const uint2 e = sym[t->lo[s] ^ 0x80u];  // any byte of range s carries its bias/start
+        const uint32_t X = L + slot;
+        const uint32_t nb = (X + e.x) >> 16;
+        v = ((uint32_t)enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)] - L) | (nb << 12);
+      }
+      for (uint32_t c = 0; c < rep; ++c) T[i * rep + c] = (uint16_t)v;
+    }
+    sc.B = B;
+    sc.T = T;
+    sc.R = R;
+    sc.rep_shift = 31u - __clz(rep);
+    sc.brep = lane & (kByteReplicas - 1);
+    sc.trep = lane & (rep - 1);
+  } else {
+    uint2* s2 = reinterpret_cast<uint2*>(smem);
+    uint16_t* e2 = reinterpret_cast<uint16_t*>(smem + 256 * 8);
+    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s2[i] = sym[i];
+    for (uint32_t i = threadIdx.x; i < L; i += blockDim.x) e2[i] = enc[i];
+    rc.sym = s2;
+    rc.enc = e2;
+    rc.L = L;
+  }
+}
+
+// Run one chunk backwards (FORMAT.md §6-§7), calling sink(field, width) for every field. seg points
+// at the segment's first byte; the chunk's symbols are its pieces in order, so the last piece is
+// coded first. Full pieces are 16-byte loads, which a warp's 32 chunks of one group issue as 512
+// consecutive bytes.
+template <int S, class Coder, class Sink>
+__device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, const ChunkGeo& g, uint32_t* st,
+                                           uint32_t& flags, Sink& sink) {
   int k = (int)g.pieces - 1;
   if (g.last_len < 16) {  // the group's short last piece, symbol by symbol
     const uint8_t* src = seg + g.base + 16u * (g.j + (uint32_t)k * g.m);
     for (int t = (int)g.last_len - 1; t >= 0; --t) {
       const int q = t & (S - 1);  // chunk index 16k + t, and S divides 16
-      uint32_t Xq = X[0];
+      uint32_t x = st[0];
 #pragma unroll
       for (int z = 1; z < S; ++z)
-        if (z == q) Xq = X[z];
+        if (z == q) x = st[z];
       uint32_t w;
-      const uint32_t field = enc_step(sm, src[t], Xq, w, flags);
+      const uint32_t field = cd.step(src[t], x, w, flags);
 #pragma unroll
       for (int z = 0; z < S; ++z)
-        if (z == q) X[z] = Xq;
-      bits += w;
-      if (WRITE) ww->put(field, w);
+        if (z == q) st[z] = x;
+      sink(field, w);
     }
     --k;
+    sink.piece_done();
   }
   const bool aligned = ((reinterpret_cast<uintptr_t>(seg + g.base) & 15u) == 0);
   for (; k >= 0; --k) {
@@ -120,73 +193,138 @@ __device__ __forceinline__ void encode_chunk(const EncSmem& sm, const uint8_t* s
     }
 #pragma unroll
     for (int r = 15; r >= 0; --r) {
-      const uint32_t b = (wv[r >> 2] >> (8 * (r & 3))) & 0xFFu;
+      const uint32_t b = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
       uint32_t w;
-      const uint32_t field = enc_step(sm, b, X[r & (S - 1)], w, flags);
-      bits += w;
-      if (WRITE) ww->put(field, w);
+      const uint32_t field = cd.step(b, st[r & (S - 1)], w, flags);
+      sink(field, w);
     }
+    sink.piece_done();
   }
-#pragma unroll
-  for (int q = 0; q < S; ++q) {
-    if (WRITE) ww->put(X[q] - L, R);
-  }
-  bits_out = bits;
 }
 
-template <int S>
+struct BitCounter {
+  uint64_t bits = 0;
+  __device__ __forceinline__ void operator()(uint32_t, uint32_t w) { bits += w; }
+  __device__ __forceinline__ void piece_done() {}
+};
+
+// Write-pass sink: LSB-first bit accumulator; complete words go to a per-thread ring in shared
+// memory, and whole 16-byte-aligned groups of 4 words leave it as one 16-byte store.
+struct RingWriter {
+  uint32_t* ring;     // this thread's row
+  uint32_t* payload;  // stream payload, 16-byte aligned
+  uint32_t wp, fp, end;  // next word to append, next word to store, end of this chunk (payload words)
+  unsigned long long acc;
+  uint32_t cnt;
+  __device__ __forceinline__ void operator()(uint32_t v, uint32_t n) {
+    acc |= (unsigned long long)v << cnt;
+    cnt += n;
+    if (cnt >= 32) {
+      ring[wp & (kRingWords - 1)] = (uint32_t)acc;
+      ++wp;
+      acc >>= 32;
+      cnt -= 32;
+    }
+  }
+  __device__ __forceinline__ void piece_done() {
+    while ((fp & 3u) != 0 && fp < wp) {  // unaligned head of the chunk
+      if (fp < end) payload[fp] = ring[fp & (kRingWords - 1)];
+      ++fp;
+    }
+    while (fp + 4 <= wp) {
+      if (fp + 4 <= end)
+        *reinterpret_cast<uint4*>(payload + fp) = *reinterpret_cast<const uint4*>(ring + (fp & (kRingWords - 1)));
+      fp += 4;
+    }
+  }
+  __device__ __forceinline__ void finish() {
+    if (cnt > 0) {
+      ring[wp & (kRingWords - 1)] = (uint32_t)acc;
+      ++wp;
+    }
+    piece_done();
+    for (; fp < wp; ++fp)
+      if (fp < end) payload[fp] = ring[fp & (kRingWords - 1)];
+  }
+};
+
+template <int S, bool STEP>
 __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t* __restrict__ in,
                                                                    const __grid_constant__ EncBatch b,
                                                                    const shn_table* __restrict__ tables,
                                                                    const EncodeLayout lay, EncodeWork w) {
-  __shared__ EncSmem sm;
+  extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  const uint32_t L = 1u << lay.R;
-  load_tables(sm, t, L);
+  StepCoder sc;
+  RangeCoder rc;
+  load_coder<STEP>(esm, t, lay.K, lay.R, sc, rc);
   __syncthreads();
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
-  const uint32_t nch = (uint32_t)n_chunks(len_seg, lay.C);
-  if (c >= nch) return;
+  if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
-  uint64_t bits = 0;
+  uint32_t st[S];
   uint32_t flags = 0;
-  encode_chunk<S, false>(sm, in + b.offset[seg], geo, L, lay.R, bits, flags, nullptr);
-  const uint64_t total = bits + (uint64_t)S * lay.R + 1;
+  BitCounter bc;
+  if (STEP) {
+#pragma unroll
+    for (int q = 0; q < S; ++q) st[q] = sc.init_state(0);
+    code_chunk<S>(sc, in + b.offset[seg], geo, st, flags, bc);
+  } else {
+#pragma unroll
+    for (int q = 0; q < S; ++q) st[q] = rc.init_state(0);
+    code_chunk<S>(rc, in + b.offset[seg], geo, st, flags, bc);
+  }
+  const uint64_t total = bc.bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
   if ((flags & 0x80000000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
 }
 
-template <int S>
+template <int S, bool STEP>
 __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t* __restrict__ in,
                                                                    const __grid_constant__ EncBatch b,
                                                                    const shn_table* __restrict__ tables,
                                                                    const EncodeLayout lay, EncodeWork w,
                                                                    uint8_t* __restrict__ out) {
   if (*(volatile uint32_t*)&w.status->status != 0) return;
-  __shared__ EncSmem sm;
+  extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  const uint32_t L = 1u << lay.R;
-  load_tables(sm, t, L);
+  StepCoder sc;
+  RangeCoder rc;
+  load_coder<STEP>(esm, t, lay.K, lay.R, sc, rc);
   __syncthreads();
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
-  const uint32_t nch = (uint32_t)n_chunks(len_seg, lay.C);
-  if (c >= nch) return;
+  if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
-  WordWriter ww;
-  ww.out = reinterpret_cast<uint32_t*>(out + lay.payload_offset) + w.word_offset[g];
-  ww.end = reinterpret_cast<uint32_t*>(out + lay.payload_offset) + w.word_offset[g + 1];
-  ww.acc = 0;
-  ww.cnt = 0;
-  uint64_t bits = 0;
+  RingWriter rw;
+  rw.ring = reinterpret_cast<uint32_t*>(esm + round_up(enc_table_smem_bytes(lay.K, lay.R), 16)) +
+            threadIdx.x * kRingStride;
+  rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
+  rw.wp = rw.fp = (uint32_t)w.word_offset[g];
+  rw.end = (uint32_t)w.word_offset[g + 1];
+  rw.acc = 0;
+  rw.cnt = 0;
+  uint32_t st[S];
   uint32_t flags = 0;
-  encode_chunk<S, true>(sm, in + b.offset[seg], geo, L, lay.R, bits, flags, &ww);
-  ww.put(1u, 1u);  // sentinel
-  if (ww.cnt > 0 && ww.out < ww.end) *ww.out = (uint32_t)ww.acc;
+  if (STEP) {
+#pragma unroll
+    for (int q = 0; q < S; ++q) st[q] = sc.init_state(0);
+    code_chunk<S>(sc, in + b.offset[seg], geo, st, flags, rw);
+#pragma unroll
+    for (int q = 0; q < S; ++q) rw(sc.final_bits(st[q]), lay.R);
+  } else {
+#pragma unroll
+    for (int q = 0; q < S; ++q) st[q] = rc.init_state(0);
+    code_chunk<S>(rc, in + b.offset[seg], geo, st, flags, rw);
+#pragma unroll
+    for (int q = 0; q < S; ++q) rw(rc.final_bits(st[q]), lay.R);
+  }
+  rw(1u, 1u);  // sentinel
+  rw.finish();
 }
 
 // ---- exclusive scan of the chunk word counts (3 small kernels, no inter-block waits) ----------
@@ -347,28 +485,49 @@ __global__ void encode_header_kernel(const __grid_constant__ EncBatch b, const s
   st32(out + lay.index_offset + 4 * g, (uint32_t)(w.word_offset[g] - w.word_offset[b.first_chunk[lo]]));
 }
 
-template <int S>
+template <int S, bool STEP>
 static cudaError_t launch_sizes_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, cudaStream_t s) {
-  encode_sizes_kernel<S><<<b.total_blocks, kEncThreads, 0, s>>>(d_in, b, d_tables, lay, w);
+  const size_t smem = enc_table_smem_bytes(lay.K, lay.R);
+  cudaError_t e = cudaFuncSetAttribute(encode_sizes_kernel<S, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  encode_sizes_kernel<S, STEP><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w);
   return cudaGetLastError();
 }
-template <int S>
+template <int S, bool STEP>
 static cudaError_t launch_write_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
-  encode_write_kernel<S><<<b.total_blocks, kEncThreads, 0, s>>>(d_in, b, d_tables, lay, w, d_out);
+  const size_t smem = round_up(enc_table_smem_bytes(lay.K, lay.R), 16) + kEncThreads * kRingStride * 4;
+  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  encode_write_kernel<S, STEP><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
   return cudaGetLastError();
+}
+
+template <int S>
+static cudaError_t sizes_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
+                                  const EncodeWork& w, cudaStream_t s) {
+  return step_replicas(lay.K, lay.R) ? launch_sizes_t<S, true>(d_in, b, t, lay, w, s)
+                                     : launch_sizes_t<S, false>(d_in, b, t, lay, w, s);
+}
+template <int S>
+static cudaError_t write_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
+                                  const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
+  return step_replicas(lay.K, lay.R) ? launch_write_t<S, true>(d_in, b, t, lay, w, d_out, s)
+                                     : launch_write_t<S, false>(d_in, b, t, lay, w, d_out, s);
 }
 
 cudaError_t launch_encode_sizes(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                 const EncodeLayout& lay, const EncodeWork& w, int, cudaStream_t s) {
   if (b.total_blocks == 0) return cudaSuccess;
   switch (lay.S) {
-    case 1: return launch_sizes_t<1>(d_in, b, d_tables, lay, w, s);
-    case 2: return launch_sizes_t<2>(d_in, b, d_tables, lay, w, s);
-    case 4: return launch_sizes_t<4>(d_in, b, d_tables, lay, w, s);
-    case 8: return launch_sizes_t<8>(d_in, b, d_tables, lay, w, s);
-    case 16: return launch_sizes_t<16>(d_in, b, d_tables, lay, w, s);
+    case 1: return sizes_dispatch<1>(d_in, b, d_tables, lay, w, s);
+    case 2: return sizes_dispatch<2>(d_in, b, d_tables, lay, w, s);
+    case 4: return sizes_dispatch<4>(d_in, b, d_tables, lay, w, s);
+    case 8: return sizes_dispatch<8>(d_in, b, d_tables, lay, w, s);
+    case 16: return sizes_dispatch<16>(d_in, b, d_tables, lay, w, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -378,11 +537,11 @@ cudaError_t launch_encode_write(const uint8_t* d_in, const EncBatch& b, const sh
                                 cudaStream_t s) {
   if (b.total_blocks == 0) return cudaSuccess;
   switch (lay.S) {
-    case 1: return launch_write_t<1>(d_in, b, d_tables, lay, w, d_out, s);
-    case 2: return launch_write_t<2>(d_in, b, d_tables, lay, w, d_out, s);
-    case 4: return launch_write_t<4>(d_in, b, d_tables, lay, w, d_out, s);
-    case 8: return launch_write_t<8>(d_in, b, d_tables, lay, w, d_out, s);
-    case 16: return launch_write_t<16>(d_in, b, d_tables, lay, w, d_out, s);
+    case 1: return write_dispatch<1>(d_in, b, d_tables, lay, w, d_out, s);
+    case 2: return write_dispatch<2>(d_in, b, d_tables, lay, w, d_out, s);
+    case 4: return write_dispatch<4>(d_in, b, d_tables, lay, w, d_out, s);
+    case 8: return write_dispatch<8>(d_in, b, d_tables, lay, w, d_out, s);
+    case 16: return write_dispatch<16>(d_in, b, d_tables, lay, w, d_out, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -140,6 +140,7 @@ int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params
  *  d_out_bytes   device uint64: the stream size in bytes (written even when it exceeds the
  *                capacity, in which case the device status is SHN_ERR_CAPACITY and d_out holds
  *                no complete stream).
+ * Streams whose shn_encode_bound exceeds 16 GiB are rejected with SHN_ERR_INVALID_ARG.
  * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_WORKSPACE, SHN_ERR_CUDA; device: SHN_ERR_CAPACITY,
  *         SHN_ERR_INVALID_ARG (a table with bad status or a symbol absent from its table).
  */
