@@ -28,9 +28,16 @@
 // chunk, and a decoded next-state row is always inside the table by construction.
 #include "shn_internal.cuh"
 
+#ifndef DEC_WARPS
+#define DEC_WARPS 4  // warps per block (tile = 32 * DEC_WARPS chunks)
+#endif
+#ifndef DEC_MIN_BLOCKS
+#define DEC_MIN_BLOCKS (32 / DEC_WARPS)  // blocks per SM the register budget must allow (<= 64 regs)
+#endif
+
 namespace shn {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = DEC_WARPS;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr uint32_t kRingQuads = 8;                // 16-byte quads per thread
 constexpr uint32_t kRingBytes = kRingQuads * 16;  // per thread
@@ -142,13 +149,15 @@ __host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
   const uint32_t L = 1u << R;
   l.table_bytes = L * kReplicas * 8;
   l.ring_off = l.table_bytes;
-  l.stage_off = l.ring_off + kDecThreads * kRingBytes;
+  // table builds happen only while no chunk is being decoded (rings idle, no copies in flight),
+  // so the build staging area shares the rings' space
+  l.stage_off = l.ring_off;
   l.stage_per_table = (uint32_t)round_up(2 * (K + 1) + 2 * K + 4 * K, 16);
   uint32_t by_table = l.table_bytes / (L * 8);
   uint32_t by_stage = kStageBytes / l.stage_per_table;
   l.max_plain_tables = by_table < by_stage ? by_table : by_stage;
   if (l.max_plain_tables < 1) l.max_plain_tables = 1;
-  l.total = l.stage_off + kStageBytes;
+  l.total = l.ring_off + (kDecThreads * kRingBytes > kStageBytes ? kDecThreads * kRingBytes : kStageBytes);
   return l;
 }
 
@@ -269,6 +278,18 @@ struct Fetcher {
       cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
     }
   }
+  // Per 16-symbol piece at most 2 quads (256 bits, the most 16 fields of <= 16 bits can use) leave
+  // the ring, so topping it up with at most 2 fetches keeps it full: no loop, two predicated copies.
+  __device__ __forceinline__ void top_up2(const ChunkCtx& c, int32_t limit) {
+    const int32_t target = limit > bottom ? limit : bottom;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (lo > target) {
+        --lo;
+        cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
+      }
+    }
+  }
 };
 
 template <int S, int SH>
@@ -314,7 +335,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
   const uint32_t full = c.pieces - (c.last_len < 16 ? 1u : 0u);
   uint8_t* dst = c.dst;
   for (uint32_t k = 0; k < full; ++k, dst += c.dst_stride) {
-    fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    fe.top_up2(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<1>();
     uint32_t ov[4];
@@ -395,7 +416,7 @@ __device__ __forceinline__ uint32_t segment_of(const uint8_t* descs, uint32_t n_
 }
 
 template <int S>
-__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const uint8_t* __restrict__ comp, DeviceStatus* st,
+__global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(const uint8_t* __restrict__ comp, DeviceStatus* st,
                                                              uint8_t* __restrict__ out) {
   extern __shared__ __align__(128) unsigned char dsm[];
   if (*(volatile uint32_t*)&st->status != 0) return;

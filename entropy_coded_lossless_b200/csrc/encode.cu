@@ -13,8 +13,10 @@
 //
 // Shared-memory tables. Each block codes chunks of one segment. When the (range, state) product
 // fits, the block expands the segment's table into one step table
-//   T[s][slot] = next slot | nb << 12     (nb = renormalisation bits of state L + slot for range s)
-// and a byte table B[b] = s | w << 8 | offset << 16 | absent << 31, both stored several times
+//   T[s][slot] = next slot | (nb + w) << 8 | (r << w) << 13
+// (nb = renormalisation bits of state L + slot for range s, r = its low nb bits, w = the range's
+// offset width; the field is then offset | r << w) and a byte table B[b] = offset | s << 8 |
+// absent << 31, both stored several times
 // interleaved ([entry][replica], replica from the lane index) so that a warp's lookups spread over
 // the banks instead of colliding. Otherwise it keeps Algorithm 2's per-range bias/start form.
 #include "shn_internal.cuh"
@@ -22,15 +24,17 @@
 namespace shn {
 
 constexpr int kEncThreads = 128;
-constexpr uint32_t kByteReplicas = 4;
-constexpr uint32_t kStepTableBudget = 16384;  // bytes of shared memory for the replicated T
-constexpr uint32_t kRingWords = 32;           // per-thread output staging ring (write pass)
-constexpr uint32_t kRingStride = kRingWords + 4;  // 144-byte rows: 16-byte reads of 8 rows hit distinct banks
+constexpr uint32_t kByteReplicas = 8;
+constexpr uint32_t kStepTableBudget = 32768;  // bytes of shared memory for the replicated T
+constexpr uint32_t kRingWords = 16;           // per-thread output staging ring (write pass)
+constexpr uint32_t kRingStride = kRingWords + 4;  // 80-byte rows: 16-byte reads of 8 rows hit distinct banks
 
+// Step-table form: L <= 256 (fields <= 16 bits, next slot in 8 bits) and the table fits.
 __host__ __device__ inline uint32_t step_replicas(uint32_t K, uint32_t R) {
-  const uint32_t bytes = K * (1u << R) * 2u;
+  if (R > 8) return 0;
+  const uint32_t bytes = K * (1u << R) * 4u;
   if (bytes > kStepTableBudget) return 0;  // step table does not fit: per-range form
-  uint32_t r = 8;
+  uint32_t r = 4;
   while (r > 1 && bytes * r > kStepTableBudget) r >>= 1;
   return r;
 }
@@ -48,25 +52,23 @@ __device__ __forceinline__ int block_segment(const EncBatch& b) {
 
 // ---- the two table forms ---------------------------------------------------------------------
 
-// Replicated step table form. State is the slot X - L.
+// Replicated step table form (L <= 256). State is the slot X - L.
 struct StepCoder {
   const uint32_t* B;   // [256][kByteReplicas]
-  const uint16_t* T;   // [K*L][rep]
+  const uint32_t* T;   // [K*L][rep]
   uint32_t R, rep_shift, brep, trep;
+  static constexpr bool kPairs = true;  // fields are <= 16 bits: two fit one 32-bit append
   __device__ __forceinline__ uint32_t init_state(uint32_t) const { return 0u; }
   __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st; }  // X - L
   // one symbol: returns the field (offset low, state bits high), its width, the new state
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& st, uint32_t& width, uint32_t& flags) const {
-    const uint32_t e = B[(b << 2) + brep];
-    const uint32_t sidx = ((e & 0xFFu) << R) | st;
+    const uint32_t e = B[b * kByteReplicas + brep];
+    const uint32_t sidx = (__byte_perm(e, 0u, 0x4441u) << R) | st;
     const uint32_t tv = T[(sidx << rep_shift) + trep];
-    const uint32_t nb = tv >> 12;
-    const uint32_t w = (e >> 8) & 0xFu;
-    const uint32_t r = st & ~(0xFFFFFFFFu << nb);
     flags |= e;
-    st = tv & 0xFFFu;
-    width = w + nb;
-    return ((e >> 16) & 0xFFu) | (r << w);
+    st = tv & 0xFFu;
+    width = (tv >> 8) & 31u;
+    return (tv >> 13) | (e & 0xFFu);
   }
 };
 
@@ -75,6 +77,7 @@ struct RangeCoder {
   const uint2* sym;
   const uint16_t* enc;
   uint32_t L;
+  static constexpr bool kPairs = false;
   __device__ __forceinline__ uint32_t init_state(uint32_t) const { return L; }
   __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st - L; }
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
@@ -92,7 +95,7 @@ struct RangeCoder {
 
 __host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t K, uint32_t R) {
   const uint32_t rep = step_replicas(K, R);
-  if (rep) return 256 * kByteReplicas * 4 + K * (1u << R) * 2 * rep;
+  if (rep) return 256 * kByteReplicas * 4 + K * (1u << R) * 4 * rep;
   return 256 * 8 + (1u << R) * 2;
 }
 
@@ -107,7 +110,7 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   if (STEP) {
     const uint32_t rep = step_replicas(K, R);
     uint32_t* B = reinterpret_cast<uint32_t*>(smem);
-    uint16_t* T = reinterpret_cast<uint16_t*>(smem + 256 * kByteReplicas * 4);
+    uint32_t* T = reinterpret_cast<uint32_t*>(smem + 256 * kByteReplicas * 4);
     for (uint32_t b = threadIdx.x; b < 256; b += blockDim.x) {
       const uint32_t u = b ^ 0x80u;
       int lo = 0, hi = (int)K - 1;  // range of u: largest k with lo[k] <= u
@@ -116,8 +119,8 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
         if (t->lo[m] <= u) lo = m;
         else hi = m - 1;
       }
-      const uint32_t e = sym[b].y;  // offset and width as the record stores them
-      const uint32_t v = (uint32_t)lo | (((e >> 24) & 15u) << 8) | (((e >> 16) & 0xFFu) << 16) | (e & 0x80000000u);
+      const uint32_t e = sym[b].y;  // offset as the record stores it, and the absent flag
+      const uint32_t v = ((e >> 16) & 0xFFu) | ((uint32_t)lo << 8) | (e & 0x80000000u);
 #pragma unroll
       for (uint32_t c = 0; c < kByteReplicas; ++c) B[b * kByteReplicas + c] = v;
     }
@@ -128,9 +131,11 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
         const uint2 e = sym[t->lo[s] ^ 0x80u];  // any byte of range s carries its bias/start
         const uint32_t X = L + slot;
         const uint32_t nb = (X + e.x) >> 16;
-        v = ((uint32_t)enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)] - L) | (nb << 12);
+        const uint32_t w = (e.y >> 24) & 15u;
+        const uint32_t r = X & ((1u << nb) - 1u);
+        v = ((uint32_t)enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)] - L) | ((nb + w) << 8) | ((r << w) << 13);
       }
-      for (uint32_t c = 0; c < rep; ++c) T[i * rep + c] = (uint16_t)v;
+      for (uint32_t c = 0; c < rep; ++c) T[i * rep + c] = v;
     }
     sc.B = B;
     sc.T = T;
@@ -191,12 +196,24 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
         wv[z] = (uint32_t)src[4 * z] | ((uint32_t)src[4 * z + 1] << 8) | ((uint32_t)src[4 * z + 2] << 16) |
                 ((uint32_t)src[4 * z + 3] << 24);
     }
+    if (Coder::kPairs) {  // symbols r and r-1: their fields (<= 16 bits each) as one append
 #pragma unroll
-    for (int r = 15; r >= 0; --r) {
-      const uint32_t b = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
-      uint32_t w;
-      const uint32_t field = cd.step(b, st[r & (S - 1)], w, flags);
-      sink(field, w);
+      for (int r = 15; r >= 1; r -= 2) {
+        const uint32_t b1 = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
+        const uint32_t b2 = __byte_perm(wv[(r - 1) >> 2], 0u, 0x4440u + (uint32_t)((r - 1) & 3));
+        uint32_t w1, w2;
+        const uint32_t f1 = cd.step(b1, st[r & (S - 1)], w1, flags);
+        const uint32_t f2 = cd.step(b2, st[(r - 1) & (S - 1)], w2, flags);
+        sink(f1 | (f2 << w1), w1 + w2);
+      }
+    } else {
+#pragma unroll
+      for (int r = 15; r >= 0; --r) {
+        const uint32_t b = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
+        uint32_t w;
+        const uint32_t field = cd.step(b, st[r & (S - 1)], w, flags);
+        sink(field, w);
+      }
     }
     sink.piece_done();
   }
@@ -214,15 +231,18 @@ struct RingWriter {
   uint32_t* ring;     // this thread's row
   uint32_t* payload;  // stream payload, 16-byte aligned
   uint32_t wp, fp, end;  // next word to append, next word to store, end of this chunk (payload words)
-  unsigned long long acc;
+  uint32_t a0, a1;    // accumulated bits: a0 holds cnt (< 32) bits, a1 the overflow of the last append
   uint32_t cnt;
+  // append the low n (<= 32) bits of v; the caller guarantees v < 2^n
   __device__ __forceinline__ void operator()(uint32_t v, uint32_t n) {
-    acc |= (unsigned long long)v << cnt;
+    a0 |= v << cnt;
+    a1 |= __funnelshift_l(v, 0u, cnt);  // bits of v beyond position 32 (none when cnt == 0)
     cnt += n;
     if (cnt >= 32) {
-      ring[wp & (kRingWords - 1)] = (uint32_t)acc;
+      ring[wp & (kRingWords - 1)] = a0;
       ++wp;
-      acc >>= 32;
+      a0 = a1;
+      a1 = 0;
       cnt -= 32;
     }
   }
@@ -239,7 +259,7 @@ struct RingWriter {
   }
   __device__ __forceinline__ void finish() {
     if (cnt > 0) {
-      ring[wp & (kRingWords - 1)] = (uint32_t)acc;
+      ring[wp & (kRingWords - 1)] = a0;
       ++wp;
     }
     piece_done();
@@ -306,7 +326,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
   rw.wp = rw.fp = (uint32_t)w.word_offset[g];
   rw.end = (uint32_t)w.word_offset[g + 1];
-  rw.acc = 0;
+  rw.a0 = 0;
+  rw.a1 = 0;
   rw.cnt = 0;
   uint32_t st[S];
   uint32_t flags = 0;
