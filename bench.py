@@ -36,22 +36,34 @@ UNIT = "GB/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="kv", choices=["kv", "weight", "sweep", "activations"])
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
+    ap.add_argument("--profile-only", action="store_true",
+                    help="run compress + decode twice untimed and exit (the case profiles/ captures)")
     return ap.parse_args()
 
 
-def workload(name, device, seed_offset=0):
+def workload(name, device, seed_offset=0, n_segments=0):
     """(int8 tensor, segments, params dict, description)."""
     if name == "kv":
-        x = inputs.kv_cache_int8(seed=2 + seed_offset, device=device)
         segs = inputs.kv_cache_segments()
-        desc = "kv_cache_int8[32,2,8,8,4096,128] (2 GiB, 64 segments = layer x K/V)"
+        if n_segments and n_segments < len(segs):
+            seg = segs[0][1]
+            segs = segs[:n_segments]
+            x = torch.empty(n_segments * seg, dtype=torch.int8, device=device)
+            for i in range(n_segments):
+                x[i * seg:(i + 1) * seg] = inputs.kv_cache_segment_int8(i // 2, i % 2, seed=2 + seed_offset,
+                                                                        device=device)
+            desc = f"kv_cache_int8 first {n_segments} of 64 layer x K/V segments ({n_segments * seg} bytes)"
+        else:
+            x = inputs.kv_cache_int8(seed=2 + seed_offset, device=device)
+            desc = "kv_cache_int8[32,2,8,8,4096,128] (2 GiB, 64 segments = layer x K/V)"
     elif name == "weight":
         x = inputs.weight_like_int8(seed=1 + seed_offset, device=device)
         segs = [(0, x.numel())]
@@ -66,6 +78,67 @@ def workload(name, device, seed_offset=0):
     return x, segs, dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4), desc
 
 
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank codes its own bytes_per_rank each step; time is the max over ranks."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
+# DRAM bytes (read + write) per symbol of each kernel, from the ncu captures summarised in
+# profiles/<kernel>_kv_cache_1GiB.md (KV cache, K=16, L=128, C=4096, S=4), with the sha256 prefix of
+# the kernel's source file at capture time: if the source has changed since, the figure is stale and
+# the bench reports traffic as null.
+MEASURED_TRAFFIC = {
+    "decode_kernel": {
+        "bytes_per_symbol": 1.8637,
+        "source": "decode.cu",
+        "sha256_prefix": "fbee812352b2843e"
+    },
+    "encode_write_kernel": {
+        "bytes_per_symbol": 1.9429,
+        "source": "encode.cu",
+        "sha256_prefix": "e69096e9fafd4ba6"
+    },
+    "encode_sizes_kernel": {
+        "bytes_per_symbol": 1.0037,
+        "source": "encode.cu",
+        "sha256_prefix": "e69096e9fafd4ba6"
+    },
+    "histogram_kernel": {
+        "bytes_per_symbol": 1.0056,
+        "source": "histogram.cu",
+        "sha256_prefix": "19a0a2a5457d1407"
+    },
+    "build_tables_kernel": {
+        "bytes_per_symbol": 0.0001,
+        "source": "build_tables.cu",
+        "sha256_prefix": "da8b40b8d15eabba"
+    }
+}
+
+
+def measured_traffic(kernels, n_symbols):
+    """Total DRAM bytes of the given kernels for n_symbols, or None if any capture is stale."""
+    import hashlib
+
+    total = 0.0
+    for k in kernels:
+        m = MEASURED_TRAFFIC[k]
+        path = os.path.join(ROOT, "entropy_coded_lossless_b200", "csrc", m["source"])
+        if hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] != m["sha256_prefix"]:
+            return None
+        total += m["bytes_per_symbol"] * n_symbols
+    return total
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -76,7 +149,7 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms; summary() covers the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -91,7 +164,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
@@ -100,7 +173,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def window(self, t0, t1):
+        """Keep only the samples taken between host times t0 and t1."""
+        self.lines = [(t, ln) for t, ln in self.lines if t0 <= t <= t1]
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -114,7 +191,7 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for _, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -264,56 +341,69 @@ def main():
                                              device_id=dev)
     from entropy_coded_lossless_b200 import shn
 
-    x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank)
+    x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank, n_segments=args.segments)
     p = shn.CodecParams(**p_dict)
     codec = shn.Codec(segs, p, device=dev)
     n = codec.n_symbols
     out = torch.empty(n, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     comp_cap = codec.stream_buf.numel()
+    if args.profile_only:
+        for _ in range(2):
+            codec.compress(x)
+            codec.decode(codec.stream_buf, comp_cap, out)
+        torch.cuda.synchronize()
+        ok = codec.status("enc")[0] == 0 and codec.status("dec")[0] == 0 and torch.equal(out, x.view(torch.uint8))
+        print(json.dumps({"profile_case": desc, "symbols": n, "stream_bytes": int(codec.out_bytes.item()),
+                          "correct": bool(ok)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        sys.exit(0 if ok else 3)
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-    stage_ms = {"histogram": 0.0, "build": 0.0, "encode": 0.0, "decode": 0.0}
+    stage_names = ("histogram", "build", "encode", "decode")
+    stage_ms = {k: 0.0 for k in stage_names}
 
-    def step(timed):
-        if timed:
-            ev[0].record(stream)
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
         codec.histogram(x)
-        if timed:
-            ev[1].record(stream)
+        if evs:
+            evs[1].record(stream)
         codec.build()
-        if timed:
-            ev[2].record(stream)
+        if evs:
+            evs[2].record(stream)
         codec.encode(x)
-        if timed:
-            ev[3].record(stream)
+        if evs:
+            evs[3].record(stream)
         codec.decode(codec.stream_buf, comp_cap, out)
-        if timed:
-            ev[4].record(stream)
-            ev[4].synchronize()
-            for i, k in enumerate(stage_ms):
-                stage_ms[k] += ev[i].elapsed_time(ev[i + 1])
+        if evs:
+            evs[4].record(stream)
 
-    for _ in range(args.warmup):
-        step(False)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # events for every timed step, read only after the last one (no host sync inside the region)
+    evs_all = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     with ClockSampler(local_rank) as clk:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0 = time.time()
         t0.record(stream)
-        for _ in range(args.steps):
-            step(True)
+        for i in range(args.steps):
+            step(evs_all[i])
         t1.record(stream)
         torch.cuda.synchronize()
+        h1 = time.time()
+        time.sleep(0.15)
+    clk.window(h0, h1)
+    for evs in evs_all:
+        for i, k in enumerate(stage_names):
+            stage_ms[k] += evs[i].elapsed_time(evs[i + 1])
     if world > 1:
         torch.distributed.barrier()
-    ms_total = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), dev)
     ms_step = ms_total / args.steps
 
     # correctness of the timed work
@@ -352,12 +442,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1) / ksteps
-        if world > 1:
-            tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(tt.item())
-        e2e = {"value": world * n / (ms_e2e * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": n,
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / ksteps, dev)
+        e2e = {"value": whole_job_gbs(n, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": n,
                "d2h_bytes_per_step": nbytes + 16, "ms_per_step": ms_e2e,
                "what": "pinned H2D input + shn_histogram + shn_build_tables + shn_encode + shn_decode + D2H stream/status"}
 
@@ -370,18 +456,21 @@ def main():
         alg = {"histogram": n, "build": 0, "encode": n + nbytes, "decode": n + nbytes}
         dom = max(("encode", "decode", "histogram"), key=lambda k: stages[k]["ms"])
 
+        kernels_of = {"decode": ["decode_kernel"], "encode": ["encode_sizes_kernel", "encode_write_kernel"],
+                      "histogram": ["histogram_kernel"]}
+
         def roof(k):
             ms = stages[k]["ms"]
             a = alg[k] / (ms * 1e-3) / 1e9
             return {"bound": "hbm", "achieved": a, "peak": peak, "unit": "GB/s", "frac": a / peak,
-                    "traffic": None, "kernel": {"decode": "decode_kernel", "encode": "encode_{sizes,write}_kernel",
-                                                "histogram": "histogram_kernel"}[k],
-                    "alg_bytes_per_launch": alg[k], "peak_kind": peak_kind}
+                    "traffic": measured_traffic(kernels_of[k], n), "kernel": "+".join(kernels_of[k]),
+                    "alg_bytes_per_launch": alg[k], "peak_kind": peak_kind,
+                    "timing": "CUDA events around the C-ABI call on the launching stream, mean over the timed steps"}
 
         launches_per_step = 1 + 1 + 1 + 3 + 1 + 1 + 2  # hist, build, sizes, scan x3, header, write, check+decode
         line = {
             "metric": METRIC,
-            "value": world * n / (ms_step * 1e-3) / 1e9,
+            "value": whole_job_gbs(n, world, ms_step),
             "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps,

@@ -11,32 +11,29 @@
 // records and chunk index are written, (4) every thread re-runs its chunk and writes the words to
 // their final place. No device-wide spin waits; everything is ordered by the stream.
 //
-// Shared-memory tables. Each block codes chunks of one segment. When the (range, state) product
-// fits, the block expands the segment's table into one step table
-//   T[s][slot] = next slot | (nb + w) << 8 | (r << w) << 13
-// (nb = renormalisation bits of state L + slot for range s, r = its low nb bits, w = the range's
-// offset width; the field is then offset | r << w) and a byte table B[b] = offset | s << 8 |
-// absent << 31, both stored several times
-// interleaved ([entry][replica], replica from the lane index) so that a warp's lookups spread over
-// the banks instead of colliding. Otherwise it keeps Algorithm 2's per-range bias/start form.
+// Shared-memory tables. Each block codes chunks of one segment and keeps Algorithm 2's per-range
+// form in shared memory: sym[raw byte] = {bias, (start + 4096) | offset << 16 | w << 24 | absent << 31}
+// and enc[L] (next state). A warp's 32 lookups use 32 unrelated indices, so both tables are stored
+// lane-interleaved: sym 16 times ([byte][16] x 8 bytes: an 8-byte load is served per half-warp, so
+// the 16 lanes of a phase always hit 16 distinct bank pairs) and enc up to 32 times ([index][copies]
+// x 2 bytes: every lane reads its own bank). Lookups are conflict-free whatever the data.
 #include "shn_internal.cuh"
 
 namespace shn {
 
 constexpr int kEncThreads = 128;
-constexpr uint32_t kByteReplicas = 8;
-constexpr uint32_t kStepTableBudget = 32768;  // bytes of shared memory for the replicated T
-constexpr uint32_t kRingWords = 16;           // per-thread output staging ring (write pass)
+constexpr uint32_t kSymCopies = 16;
+constexpr uint32_t kEncCopyBudget = 16384;        // bytes for the replicated next-state table
+constexpr uint32_t kRingWords = 16;               // per-thread output staging ring (write pass)
 constexpr uint32_t kRingStride = kRingWords + 4;  // 80-byte rows: 16-byte reads of 8 rows hit distinct banks
 
-// Step-table form: L <= 256 (fields <= 16 bits, next slot in 8 bits) and the table fits.
-__host__ __device__ inline uint32_t step_replicas(uint32_t K, uint32_t R) {
-  if (R > 8) return 0;
-  const uint32_t bytes = K * (1u << R) * 4u;
-  if (bytes > kStepTableBudget) return 0;  // step table does not fit: per-range form
-  uint32_t r = 4;
-  while (r > 1 && bytes * r > kStepTableBudget) r >>= 1;
-  return r;
+__host__ __device__ inline uint32_t enc_copies(uint32_t R) {
+  uint32_t c = 32;
+  while (c > 1 && (2u << R) * c > kEncCopyBudget) c >>= 1;
+  return c;
+}
+__host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t R) {
+  return 256 * kSymCopies * 8 + (2u << R) * enc_copies(R);
 }
 
 // Segment of this block: largest s with block_start[s] <= blockIdx.x.
@@ -50,115 +47,46 @@ __device__ __forceinline__ int block_segment(const EncBatch& b) {
   return lo;
 }
 
-// ---- the two table forms ---------------------------------------------------------------------
-
-// Replicated step table form (L <= 256). State is the slot X - L.
-struct StepCoder {
-  const uint32_t* B;   // [256][kByteReplicas]
-  const uint32_t* T;   // [K*L][rep]
-  uint32_t R, rep_shift, brep, trep;
-  static constexpr bool kPairs = true;  // fields are <= 16 bits: two fit one 32-bit append
-  __device__ __forceinline__ uint32_t init_state(uint32_t) const { return 0u; }
-  __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st; }  // X - L
-  // one symbol: returns the field (offset low, state bits high), its width, the new state
-  __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& st, uint32_t& width, uint32_t& flags) const {
-    const uint32_t e = B[b * kByteReplicas + brep];
-    const uint32_t sidx = (__byte_perm(e, 0u, 0x4441u) << R) | st;
-    const uint32_t tv = T[(sidx << rep_shift) + trep];
-    flags |= e;
-    st = tv & 0xFFu;
-    width = (tv >> 8) & 31u;
-    return (tv >> 13) | (e & 0xFFu);
-  }
-};
-
-// Per-range form (Algorithm 2's bias/start): sym[raw byte] = {bias, (start + 4096) | o << 16 | w << 24}.
-struct RangeCoder {
-  const uint2* sym;
-  const uint16_t* enc;
+// Algorithm 2 per symbol, on the lane-interleaved tables. State X in [L, 2L).
+struct Coder {
+  const unsigned char* sym;  // this lane's column: + raw byte * 128
+  const unsigned char* enc;  // this lane's column of the next-state table
+  uint32_t enc_row;          // bytes per enc index (2 * copies)
   uint32_t L;
-  static constexpr bool kPairs = false;
-  __device__ __forceinline__ uint32_t init_state(uint32_t) const { return L; }
-  __device__ __forceinline__ uint32_t final_bits(uint32_t st) const { return st - L; }
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
-    const uint2 e = sym[b];
+    const uint2 e = *reinterpret_cast<const uint2*>(sym + b * (kSymCopies * 8));
     const uint32_t nb = (X + e.x) >> 16;
     const uint32_t w = (e.y >> 24) & 15u;
-    const uint32_t o = (e.y >> 16) & 0xFFu;
-    const uint32_t r = X & ((1u << nb) - 1u);
-    X = enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)];
+    const uint32_t r = X & ~(0xFFFFFFFFu << nb);
+    X = *reinterpret_cast<const uint16_t*>(enc + ((e.y & 0xFFFFu) + (X >> nb) - 4096u) * enc_row);
     flags |= e.y;
     width = w + nb;
-    return o | (r << w);
+    return __byte_perm(e.y, 0u, 0x4442u) | (r << w);  // offset | state bits above it
   }
 };
 
-__host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t K, uint32_t R) {
-  const uint32_t rep = step_replicas(K, R);
-  if (rep) return 256 * kByteReplicas * 4 + K * (1u << R) * 4 * rep;
-  return 256 * 8 + (1u << R) * 2;
-}
-
-// Expand table record t into shared memory (all threads of the block).
-template <bool STEP>
-__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t K, uint32_t R,
-                                           StepCoder& sc, RangeCoder& rc) {
+__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t R, Coder& cd) {
   const uint32_t L = 1u << R;
+  const uint32_t copies = enc_copies(R);
   const uint2* sym = table_sym(t);
   const uint16_t* enc = table_enc(t);
+  uint2* s2 = reinterpret_cast<uint2*>(smem);
+  uint16_t* e2 = reinterpret_cast<uint16_t*>(smem + 256 * kSymCopies * 8);
+  for (uint32_t i = threadIdx.x; i < 256 * kSymCopies; i += blockDim.x) s2[i] = sym[i / kSymCopies];
+  for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x) e2[i] = enc[i / copies];
   const uint32_t lane = threadIdx.x & 31;
-  if (STEP) {
-    const uint32_t rep = step_replicas(K, R);
-    uint32_t* B = reinterpret_cast<uint32_t*>(smem);
-    uint32_t* T = reinterpret_cast<uint32_t*>(smem + 256 * kByteReplicas * 4);
-    for (uint32_t b = threadIdx.x; b < 256; b += blockDim.x) {
-      const uint32_t u = b ^ 0x80u;
-      int lo = 0, hi = (int)K - 1;  // range of u: largest k with lo[k] <= u
-      while (lo < hi) {
-        const int m = (lo + hi + 1) >> 1;
-        if (t->lo[m] <= u) lo = m;
-        else hi = m - 1;
-      }
-      const uint32_t e = sym[b].y;  // offset as the record stores it, and the absent flag
-      const uint32_t v = ((e >> 16) & 0xFFu) | ((uint32_t)lo << 8) | (e & 0x80000000u);
-#pragma unroll
-      for (uint32_t c = 0; c < kByteReplicas; ++c) B[b * kByteReplicas + c] = v;
-    }
-    for (uint32_t i = threadIdx.x; i < K * L; i += blockDim.x) {
-      const uint32_t s = i >> R, slot = i & (L - 1);
-      uint32_t v = 0;
-      if (t->f[s] != 0) {
-        const uint2 e = sym[t->lo[s] ^ 0x80u];  // any byte of range s carries its bias/start
-        const uint32_t X = L + slot;
-        const uint32_t nb = (X + e.x) >> 16;
-        const uint32_t w = (e.y >> 24) & 15u;
-        const uint32_t r = X & ((1u << nb) - 1u);
-        v = ((uint32_t)enc[(e.y & 0xFFFFu) - 4096u + (X >> nb)] - L) | ((nb + w) << 8) | ((r << w) << 13);
-      }
-      for (uint32_t c = 0; c < rep; ++c) T[i * rep + c] = v;
-    }
-    sc.B = B;
-    sc.T = T;
-    sc.R = R;
-    sc.rep_shift = 31u - __clz(rep);
-    sc.brep = lane & (kByteReplicas - 1);
-    sc.trep = lane & (rep - 1);
-  } else {
-    uint2* s2 = reinterpret_cast<uint2*>(smem);
-    uint16_t* e2 = reinterpret_cast<uint16_t*>(smem + 256 * 8);
-    for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) s2[i] = sym[i];
-    for (uint32_t i = threadIdx.x; i < L; i += blockDim.x) e2[i] = enc[i];
-    rc.sym = s2;
-    rc.enc = e2;
-    rc.L = L;
-  }
+  cd.sym = smem + (lane & (kSymCopies - 1)) * 8;
+  cd.enc_row = 2 * copies;
+  // entry e of copy c is at e2 + (e * copies + c) * 2
+  cd.enc = reinterpret_cast<const unsigned char*>(e2) + (lane & (copies - 1)) * 2;
+  cd.L = L;
 }
 
 // Run one chunk backwards (FORMAT.md §6-§7), calling sink(field, width) for every field. seg points
 // at the segment's first byte; the chunk's symbols are its pieces in order, so the last piece is
 // coded first. Full pieces are 16-byte loads, which a warp's 32 chunks of one group issue as 512
 // consecutive bytes.
-template <int S, class Coder, class Sink>
+template <int S, bool PAIRS, class Sink>
 __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, const ChunkGeo& g, uint32_t* st,
                                            uint32_t& flags, Sink& sink) {
   int k = (int)g.pieces - 1;
@@ -181,22 +109,28 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
     sink.piece_done();
   }
   const bool aligned = ((reinterpret_cast<uintptr_t>(seg + g.base) & 15u) == 0);
-  for (; k >= 0; --k) {
-    const uint8_t* src = seg + g.base + 16u * (g.j + (uint32_t)k * g.m);
-    uint32_t wv[4];
-    if (aligned) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
-      wv[0] = v.x;
-      wv[1] = v.y;
-      wv[2] = v.z;
-      wv[3] = v.w;
-    } else {
+  const uint8_t* piece0 = seg + g.base + 16u * g.j;
+  const uint32_t stride = 16u * g.m;
+  auto load_piece = [&](int kk) -> uint4 {
+    const uint8_t* src = piece0 + (uint32_t)kk * stride;
+    if (aligned) return __ldcs(reinterpret_cast<const uint4*>(src));
+    uint32_t v[4];
 #pragma unroll
-      for (int z = 0; z < 4; ++z)
-        wv[z] = (uint32_t)src[4 * z] | ((uint32_t)src[4 * z + 1] << 8) | ((uint32_t)src[4 * z + 2] << 16) |
-                ((uint32_t)src[4 * z + 3] << 24);
-    }
-    if (Coder::kPairs) {  // symbols r and r-1: their fields (<= 16 bits each) as one append
+    for (int z = 0; z < 4; ++z)
+      v[z] = (uint32_t)src[4 * z] | ((uint32_t)src[4 * z + 1] << 8) | ((uint32_t)src[4 * z + 2] << 16) |
+             ((uint32_t)src[4 * z + 3] << 24);
+    return make_uint4(v[0], v[1], v[2], v[3]);
+  };
+  // the next two pieces are always in flight while one is coded (loads are issued 2 pieces ahead)
+  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = make_uint4(0, 0, 0, 0);
+  if (k >= 0) p0 = load_piece(k);
+  if (k >= 1) p1 = load_piece(k - 1);
+  for (; k >= 0; --k) {
+    const uint4 cur = p0;
+    p0 = p1;
+    if (k >= 2) p1 = load_piece(k - 2);
+    const uint32_t wv[4] = {cur.x, cur.y, cur.z, cur.w};
+    if (PAIRS) {  // symbols r and r-1: their fields (<= 16 bits each, L <= 256) as one append
 #pragma unroll
       for (int r = 15; r >= 1; r -= 2) {
         const uint32_t b1 = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
@@ -220,7 +154,7 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
 }
 
 struct BitCounter {
-  uint64_t bits = 0;
+  uint32_t bits = 0;  // a chunk has at most 65536 fields of <= 20 bits
   __device__ __forceinline__ void operator()(uint32_t, uint32_t w) { bits += w; }
   __device__ __forceinline__ void piece_done() {}
 };
@@ -268,7 +202,7 @@ struct RingWriter {
   }
 };
 
-template <int S, bool STEP>
+template <int S, bool PAIRS>
 __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t* __restrict__ in,
                                                                    const __grid_constant__ EncBatch b,
                                                                    const shn_table* __restrict__ tables,
@@ -276,32 +210,25 @@ __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t
   extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  StepCoder sc;
-  RangeCoder rc;
-  load_coder<STEP>(esm, t, lay.K, lay.R, sc, rc);
+  Coder cd;
+  load_coder(esm, t, lay.R, cd);
   __syncthreads();
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   uint32_t st[S];
+#pragma unroll
+  for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
   BitCounter bc;
-  if (STEP) {
-#pragma unroll
-    for (int q = 0; q < S; ++q) st[q] = sc.init_state(0);
-    code_chunk<S>(sc, in + b.offset[seg], geo, st, flags, bc);
-  } else {
-#pragma unroll
-    for (int q = 0; q < S; ++q) st[q] = rc.init_state(0);
-    code_chunk<S>(rc, in + b.offset[seg], geo, st, flags, bc);
-  }
-  const uint64_t total = bc.bits + (uint64_t)S * lay.R + 1;
+  code_chunk<S, PAIRS>(cd, in + b.offset[seg], geo, st, flags, bc);
+  const uint64_t total = (uint64_t)bc.bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
   if ((flags & 0x80000000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
 }
 
-template <int S, bool STEP>
+template <int S, bool PAIRS>
 __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t* __restrict__ in,
                                                                    const __grid_constant__ EncBatch b,
                                                                    const shn_table* __restrict__ tables,
@@ -311,9 +238,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  StepCoder sc;
-  RangeCoder rc;
-  load_coder<STEP>(esm, t, lay.K, lay.R, sc, rc);
+  Coder cd;
+  load_coder(esm, t, lay.R, cd);
   __syncthreads();
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
@@ -321,8 +247,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
   RingWriter rw;
-  rw.ring = reinterpret_cast<uint32_t*>(esm + round_up(enc_table_smem_bytes(lay.K, lay.R), 16)) +
-            threadIdx.x * kRingStride;
+  rw.ring = reinterpret_cast<uint32_t*>(esm + round_up(enc_table_smem_bytes(lay.R), 16)) + threadIdx.x * kRingStride;
   rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
   rw.wp = rw.fp = (uint32_t)w.word_offset[g];
   rw.end = (uint32_t)w.word_offset[g + 1];
@@ -330,20 +255,12 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   rw.a1 = 0;
   rw.cnt = 0;
   uint32_t st[S];
+#pragma unroll
+  for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
-  if (STEP) {
+  code_chunk<S, PAIRS>(cd, in + b.offset[seg], geo, st, flags, rw);
 #pragma unroll
-    for (int q = 0; q < S; ++q) st[q] = sc.init_state(0);
-    code_chunk<S>(sc, in + b.offset[seg], geo, st, flags, rw);
-#pragma unroll
-    for (int q = 0; q < S; ++q) rw(sc.final_bits(st[q]), lay.R);
-  } else {
-#pragma unroll
-    for (int q = 0; q < S; ++q) st[q] = rc.init_state(0);
-    code_chunk<S>(rc, in + b.offset[seg], geo, st, flags, rw);
-#pragma unroll
-    for (int q = 0; q < S; ++q) rw(rc.final_bits(st[q]), lay.R);
-  }
+  for (int q = 0; q < S; ++q) rw(st[q] - cd.L, lay.R);
   rw(1u, 1u);  // sentinel
   rw.finish();
 }
@@ -506,38 +423,38 @@ __global__ void encode_header_kernel(const __grid_constant__ EncBatch b, const s
   st32(out + lay.index_offset + 4 * g, (uint32_t)(w.word_offset[g] - w.word_offset[b.first_chunk[lo]]));
 }
 
-template <int S, bool STEP>
+template <int S, bool PAIRS>
 static cudaError_t launch_sizes_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, cudaStream_t s) {
-  const size_t smem = enc_table_smem_bytes(lay.K, lay.R);
-  cudaError_t e = cudaFuncSetAttribute(encode_sizes_kernel<S, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = enc_table_smem_bytes(lay.R);
+  cudaError_t e = cudaFuncSetAttribute(encode_sizes_kernel<S, PAIRS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  encode_sizes_kernel<S, STEP><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w);
+  encode_sizes_kernel<S, PAIRS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w);
   return cudaGetLastError();
 }
-template <int S, bool STEP>
+template <int S, bool PAIRS>
 static cudaError_t launch_write_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
-  const size_t smem = round_up(enc_table_smem_bytes(lay.K, lay.R), 16) + kEncThreads * kRingStride * 4;
-  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = round_up(enc_table_smem_bytes(lay.R), 16) + kEncThreads * kRingStride * 4;
+  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, PAIRS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  encode_write_kernel<S, STEP><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
+  encode_write_kernel<S, PAIRS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
   return cudaGetLastError();
 }
 
+// Two fields fit one 32-bit append when they are <= 16 bits each, i.e. L <= 256.
 template <int S>
 static cudaError_t sizes_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
                                   const EncodeWork& w, cudaStream_t s) {
-  return step_replicas(lay.K, lay.R) ? launch_sizes_t<S, true>(d_in, b, t, lay, w, s)
-                                     : launch_sizes_t<S, false>(d_in, b, t, lay, w, s);
+  return lay.R <= 8 ? launch_sizes_t<S, true>(d_in, b, t, lay, w, s) : launch_sizes_t<S, false>(d_in, b, t, lay, w, s);
 }
 template <int S>
 static cudaError_t write_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
                                   const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
-  return step_replicas(lay.K, lay.R) ? launch_write_t<S, true>(d_in, b, t, lay, w, d_out, s)
-                                     : launch_write_t<S, false>(d_in, b, t, lay, w, d_out, s);
+  return lay.R <= 8 ? launch_write_t<S, true>(d_in, b, t, lay, w, d_out, s)
+                    : launch_write_t<S, false>(d_in, b, t, lay, w, d_out, s);
 }
 
 cudaError_t launch_encode_sizes(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
