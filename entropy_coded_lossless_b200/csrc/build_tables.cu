@@ -253,12 +253,12 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
     uint2 e;
     if (fs == 0) {
       e.x = 0u;  // nb = 0; enc index = X - L stays inside the table
-      e.y = (4096u - L) | (o << 16) | (w << 24) | 0x80000000u;  // absent-symbol flag
+      e.y = o | (w << 8) | 0x8000u | ((4096u - L) << 16);  // absent-symbol flag
     } else {
       const uint32_t a = 31u - __clz(fs);
       const uint32_t sh = (uint32_t)R - a;
       e.x = (sh << 16) - (fs << sh);
-      e.y = (uint32_t)((int)S.cumul[s] - (int)fs + 4096) | (o << 16) | (w << 24);
+      e.y = o | (w << 8) | ((uint32_t)((int)S.cumul[s] - (int)fs + 4096) << 16);
     }
     reinterpret_cast<uint2*>(out->opaque + kOpaqueSymOffset)[bb] = e;
     out->f[tid] = (uint16_t)S.f[tid];

@@ -58,7 +58,6 @@ EncWorkLayout enc_work_layout(uint64_t total_chunks) {
   return l;
 }
 
-constexpr int kEncBlockThreads = 128;  // chunks per encoder block (must match encode.cu)
 
 }  // namespace
 

@@ -6,12 +6,12 @@
 // backwards from its end sentinel.
 //
 // Tables. The decode table lives in shared memory as 8-byte entries
-//   .x = shared-memory offset of the next state's row (row base, including this thread's replica)
+//   .x = shared-window address of the next state's row (row base, including this thread's replica)
 //   .y = nb | w << 8 | base' << 16 | (-(nb + w) & 0xFF) << 24     (base' = range base ^ 0x80)
 // so one lookup plus two funnel shifts and one multiply-add give the next state's address. The
-// fields above bit 7 are read with multiply-high instructions (y >> s == mulhi(y, 2^(32-s)), and a
-// signed mulhi by 2^8 yields the negated field width), which run on the FMA pipe and leave the ALU
-// pipe to the funnel shifts. When a tile lies
+// fields above bit 7 are written as multiply-highs (y >> s == mulhi(y, 2^(32-s)), and a signed
+// mulhi by 2^8 yields the negated field width); the compiler chooses shift or integer-multiply
+// instructions for them (forcing the multiply pipe for all of them measured slower). When a tile lies
 // in one segment (the common case for large tensors) the table is stored 16 times interleaved
 // ([slot][replica], replica = lane & 15): an 8-byte load is served per half-warp, so the 16 lanes of
 // a half-warp always hit 16 different bank pairs whatever their states — no bank conflicts. Tiles
@@ -20,7 +20,7 @@
 //
 // Bits. Each thread keeps a 64-bit window (two words) of its chunk in registers and refills it from
 // a private 128-byte ring in shared memory, which cp.async (16-byte, L2-only) copies fill ahead of
-// use. Two symbols are extracted per window position (fields are <= 16 bits for L <= 256). Decoded
+// use. All shared-memory accesses of the per-symbol loop use 32-bit shared-window addresses. Two symbols are extracted per window position (fields are <= 16 bits for L <= 256). Decoded
 // bytes go out as 16-byte stores.
 //
 // Robustness. Corrupt input never causes an out-of-bounds access: descriptors and the chunk index
@@ -29,7 +29,7 @@
 #include "shn_internal.cuh"
 
 #ifndef DEC_WARPS
-#define DEC_WARPS 4  // warps per block (tile = 32 * DEC_WARPS chunks)
+#define DEC_WARPS 8  // warps per block (tile = 32 * DEC_WARPS chunks)
 #endif
 #ifndef DEC_MIN_BLOCKS
 #define DEC_MIN_BLOCKS (32 / DEC_WARPS)  // blocks per SM the register budget must allow (<= 64 regs)
@@ -165,7 +165,7 @@ __host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
 // slot i, replica c at byte (i*16 + c)*8; plain: table t at t*L*8, entry i at +i*8. All threads of
 // the block take part; the caller synchronises before (readers of the old tables are done).
 __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, const SmemLayout& lay, uint32_t seg0,
-                                    uint32_t nt, bool replicated, unsigned char* dsm) {
+                                    uint32_t nt, bool replicated, unsigned char* dsm, uint32_t dsm_saddr) {
   const uint32_t K = h.K, R = h.R, L = 1u << R;
   const uint32_t tid = threadIdx.x;
   for (uint32_t e = tid; e < nt * K; e += blockDim.x) {
@@ -220,9 +220,9 @@ __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, con
     if (replicated) {
       uint2* row = reinterpret_cast<uint2*>(dsm + i * (kReplicas * 8));
 #pragma unroll
-      for (uint32_t c = 0; c < kReplicas; ++c) row[c] = make_uint2(next * (kReplicas * 8) + c * 8, y);
+      for (uint32_t c = 0; c < kReplicas; ++c) row[c] = make_uint2(dsm_saddr + next * (kReplicas * 8) + c * 8, y);
     } else {
-      reinterpret_cast<uint2*>(dsm + t * L * 8)[i] = make_uint2(t * L * 8 + next * 8, y);
+      reinterpret_cast<uint2*>(dsm + t * L * 8)[i] = make_uint2(dsm_saddr + t * L * 8 + next * 8, y);
     }
   }
   __syncthreads();
@@ -239,14 +239,15 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// y >> 8, y >> 16 and the signed top byte, computed on the FMA pipe (see the file comment).
-__device__ __forceinline__ uint32_t shr8_fma(uint32_t y) { return __umulhi(y, 1u << 24); }
-__device__ __forceinline__ uint32_t add_shr16_fma(uint32_t y, uint32_t a) {
+// y >> 8, y >> 16 and the signed top byte as multiply-highs by powers of two; the compiler picks the
+// pipe (shift or integer multiply) for each.
+__device__ __forceinline__ uint32_t shr8(uint32_t y) { return __umulhi(y, 1u << 24); }
+__device__ __forceinline__ uint32_t add_shr16(uint32_t y, uint32_t a) {
   uint32_t d;
   asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(y), "r"(1u << 16), "r"(a));
   return d;
 }
-__device__ __forceinline__ int32_t add_top_byte_fma(uint32_t y, int32_t p) {  // p + (int8)(y >> 24)
+__device__ __forceinline__ int32_t add_top_byte(uint32_t y, int32_t p) {  // p + (int8)(y >> 24)
   int32_t d;
   asm("mad.hi.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(y), "r"(256), "r"(p));
   return d;
@@ -254,12 +255,10 @@ __device__ __forceinline__ int32_t add_top_byte_fma(uint32_t y, int32_t p) {  //
 
 struct ChunkCtx {
   const uint8_t* comp;
-  unsigned char* dsm;
-  uint32_t ring;        // this thread's ring: byte offset in dsm
-  uint32_t ring_saddr;  // ... as a shared-state-space address for cp.async
+  uint32_t ring_saddr;  // this thread's ring (shared-window address, 128-byte aligned)
   uint64_t cb;          // chunk start, bytes from the stream start
   uint32_t nw;          // chunk words
-  uint32_t tbase;       // offset of slot 0's entry for this thread (replica / plain table)
+  uint32_t tbase;       // shared-window address of slot 0's entry for this thread (replica / plain table)
   uint8_t* dst;         // where the chunk's first piece goes (FORMAT.md §6)
   uint32_t dst_stride;  // bytes between consecutive pieces of the chunk (16 * chunks in its group)
   uint32_t pieces;
@@ -294,7 +293,6 @@ struct Fetcher {
 
 template <int S, int SH>
 __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
-  unsigned char* const dsm = c.dsm;
   const uint32_t mask = kRingBytes - 1;
   const uint32_t cb_mod = (uint32_t)(c.cb & mask);
   Fetcher fe;
@@ -305,22 +303,21 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
   const int32_t cb_words = (int32_t)(c.cb >> 2);  // chunk start in stream words
   cp_async_commit();
   cp_async_wait<0>();
-  auto word = [&](int32_t k) -> uint32_t {  // chunk word k (k may be -1: stale, never used validly)
-    return *reinterpret_cast<const uint32_t*>(dsm + c.ring + ((cb_mod + 4u * (uint32_t)k) & mask));
-  };
-  const uint32_t last = word((int32_t)c.nw - 1);
+  // ring address of chunk word k (k may be negative: a stale word, never used validly)
+  auto waddr = [&](int32_t k) -> uint32_t { return c.ring_saddr | ((cb_mod + 4u * (uint32_t)k) & mask); };
+  const uint32_t last = lds32(waddr((int32_t)c.nw - 1));
   if (last == 0u) return false;
   int32_t P = 32 * ((int32_t)c.nw - 1) + (31 - __clz(last));  // unread bits: [0, P)
   int32_t thr = P & ~31;                                        // window = words (thr/32 - 1, thr/32)
-  uint32_t rw = (cb_mod + 4u * (uint32_t)((thr >> 5) - 1)) & mask;  // ring offset of word thr/32 - 1
-  uint32_t W1 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + ((rw + 4u) & mask));
-  uint32_t W0 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + rw);
+  uint32_t W1 = lds32(waddr((thr >> 5)));
+  uint32_t W0 = lds32(waddr((thr >> 5) - 1));
+  uint32_t ra_w = waddr((thr >> 5) - 1);  // ring address of W0
   auto advance = [&]() {  // keep P in [thr, thr + 32)
     if (P < thr) {
       W1 = W0;
       thr -= 32;
-      rw = (rw - 4u) & mask;
-      W0 = *reinterpret_cast<const uint32_t*>(dsm + c.ring + rw);
+      ra_w = c.ring_saddr | ((ra_w - 4u) & mask);
+      W0 = lds32(ra_w);
     }
   };
   uint32_t X[S];
@@ -343,23 +340,23 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
     for (int pp = 0; pp < 8; ++pp) {
       const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
       const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);  // next 32 bits, top-aligned
-      const uint2 Ea = *reinterpret_cast<const uint2*>(dsm + X[qa]);
+      const uint2 Ea = lds64(X[qa]);
       const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);          // state bits: top nb of V
       const uint32_t Va = __funnelshift_l(0u, V, Ea.y);          // V << nb
-      const uint32_t wa = shr8_fma(Ea.y);                        // low 5 bits: w
+      const uint32_t wa = shr8(Ea.y);                            // low 5 bits: w
       const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
-      const uint32_t ba = add_shr16_fma(Ea.y, oa);               // low byte: base' + offset
+      const uint32_t ba = add_shr16(Ea.y, oa);                   // low byte: base' + offset
       X[qa] = Ea.x + ra * (1u << SH);
       const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
-      P = add_top_byte_fma(Ea.y, P);                             // P -= nb + w
-      const uint2 Eb = *reinterpret_cast<const uint2*>(dsm + X[qb]);
+      P = add_top_byte(Ea.y, P);                                 // P -= nb + w
+      const uint2 Eb = lds64(X[qb]);
       const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
       const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
-      const uint32_t wb = shr8_fma(Eb.y);
+      const uint32_t wb = shr8(Eb.y);
       const uint32_t ob = __funnelshift_l(Vb, 0u, wb);
-      const uint32_t bb = add_shr16_fma(Eb.y, ob);
+      const uint32_t bb = add_shr16(Eb.y, ob);
       X[qb] = Eb.x + rb * (1u << SH);
-      P = add_top_byte_fma(Eb.y, P);
+      P = add_top_byte(Eb.y, P);
       advance();
       const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
       if ((pp & 1) == 0) ov[pp >> 1] = pair;
@@ -383,14 +380,14 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       for (int k = 1; k < S; ++k)
         if (k == q) x = X[k];
       const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
-      const uint2 E = *reinterpret_cast<const uint2*>(dsm + x);
+      const uint2 E = lds64(x);
       const uint32_t r = __funnelshift_l(V, 0u, E.y);
       const uint32_t Vs = __funnelshift_l(0u, V, E.y);
-      const uint32_t o = __funnelshift_l(Vs, 0u, shr8_fma(E.y));
+      const uint32_t o = __funnelshift_l(Vs, 0u, shr8(E.y));
       x = E.x + r * (1u << SH);
-      P = add_top_byte_fma(E.y, P);
+      P = add_top_byte(E.y, P);
       advance();
-      dst[i] = (uint8_t)add_shr16_fma(E.y, o);
+      dst[i] = (uint8_t)add_shr16(E.y, o);
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;
@@ -427,8 +424,12 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
   const uint8_t* recs = descs + (uint64_t)kSegDescBytes * h.n_segs;
   const uint32_t* index = reinterpret_cast<const uint32_t*>(comp + h.index_off);
   const uint32_t tid = threadIdx.x, lane = tid & 31;
-  const uint32_t ring = lay.ring_off + tid * kRingBytes;
-  const uint32_t ring_saddr = (uint32_t)__cvta_generic_to_shared(dsm + ring);
+  const uint32_t dsm_saddr = smem_addr(dsm);
+  const uint32_t ring_saddr = dsm_saddr + lay.ring_off + tid * kRingBytes;
+  if ((dsm_saddr & 127u) != 0) {  // ring addressing below relies on 128-byte aligned rings
+    if (tid == 0) report(st, SHN_ERR_CUDA, 0);
+    return;
+  }
   const uint64_t n_tiles = (h.total_chunks + kDecThreads - 1) / kDecThreads;
   int64_t cur_seg = -1;  // segment whose replicated table is in shared memory
 
@@ -455,8 +456,6 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
         valid = false;
       } else {
         c.comp = comp;
-        c.dsm = dsm;
-        c.ring = ring;
         c.ring_saddr = ring_saddr;
         c.cb = h.payload_off + pay_start + 4ull * w0;
         c.nw = w1 - w0;
@@ -470,11 +469,11 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
     if (sa == sb) {
       if (cur_seg != (int64_t)sa) {
         __syncthreads();
-        build_decode_tables(recs, h, lay, sa, 1, true, dsm);
+        build_decode_tables(recs, h, lay, sa, 1, true, dsm, dsm_saddr);
         cur_seg = sa;
       }
       if (valid) {
-        c.tbase = (lane & (kReplicas - 1)) * 8;
+        c.tbase = dsm_saddr + (lane & (kReplicas - 1)) * 8;
         if (!decode_chunk<S, 7>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
       }
     } else {
@@ -482,9 +481,9 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
       for (uint32_t s0 = sa; s0 <= sb; s0 += lay.max_plain_tables) {
         const uint32_t nt = min(lay.max_plain_tables, sb - s0 + 1);
         __syncthreads();
-        build_decode_tables(recs, h, lay, s0, nt, false, dsm);
+        build_decode_tables(recs, h, lay, s0, nt, false, dsm, dsm_saddr);
         if (valid && seg >= s0 && seg < s0 + nt) {
-          c.tbase = (seg - s0) * L * 8;
+          c.tbase = dsm_saddr + (seg - s0) * L * 8;
           if (!decode_chunk<S, 3>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
         }
       }

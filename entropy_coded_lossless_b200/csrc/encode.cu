@@ -21,7 +21,11 @@
 
 namespace shn {
 
-constexpr int kEncThreads = 128;
+#ifndef ENC_AHEAD
+#define ENC_AHEAD 2
+#endif
+constexpr int kEncThreads = kEncBlockThreads;
+constexpr int kEncAhead = ENC_AHEAD;  // input pieces in flight while one is coded
 constexpr uint32_t kSymCopies = 16;
 constexpr uint32_t kEncCopyBudget = 16384;        // bytes for the replicated next-state table
 constexpr uint32_t kRingWords = 16;               // per-thread output staging ring (write pass)
@@ -47,21 +51,26 @@ __device__ __forceinline__ int block_segment(const EncBatch& b) {
   return lo;
 }
 
-// Algorithm 2 per symbol, on the lane-interleaved tables. State X in [L, 2L).
+// Algorithm 2 per symbol, on the lane-interleaved tables. State X in [L, 2L). Addresses are 32-bit
+// shared-window addresses.
 struct Coder {
-  const unsigned char* sym;  // this lane's column: + raw byte * 128
-  const unsigned char* enc;  // this lane's column of the next-state table
-  uint32_t enc_row;          // bytes per enc index (2 * copies)
+  uint32_t sym;      // this lane's column of sym: + raw byte * 128
+  uint32_t enc;      // this lane's column of enc, biased by -4096 rows (the +4096 in .y's start field)
+  uint32_t enc_row;  // bytes per enc index (2 * copies)
   uint32_t L;
+  // Returns the symbol's fields (offset low, state bits above it); width = their total bit count.
+  // CHECK: accumulate .y into flags (bit 15 set for a byte absent from the table's histogram).
+  template <bool CHECK>
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
-    const uint2 e = *reinterpret_cast<const uint2*>(sym + b * (kSymCopies * 8));
+    const uint2 e = lds64(sym + b * (kSymCopies * 8));
     const uint32_t nb = (X + e.x) >> 16;
-    const uint32_t w = (e.y >> 24) & 15u;
-    const uint32_t r = X & ~(0xFFFFFFFFu << nb);
-    X = *reinterpret_cast<const uint16_t*>(enc + ((e.y & 0xFFFFu) + (X >> nb) - 4096u) * enc_row);
-    flags |= e.y;
+    const uint32_t q = X >> nb;
+    const uint32_t r = X - (q << nb);                   // the nb low state bits
+    const uint32_t w = __byte_perm(e.y, 0u, 0x4441u);  // offset width
+    X = lds_u16(enc + ((e.y >> 16) + q) * enc_row);
+    if (CHECK) flags |= e.y;
     width = w + nb;
-    return __byte_perm(e.y, 0u, 0x4442u) | (r << w);  // offset | state bits above it
+    return (r << w) | (e.y & 0xFFu);
   }
 };
 
@@ -75,10 +84,10 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   for (uint32_t i = threadIdx.x; i < 256 * kSymCopies; i += blockDim.x) s2[i] = sym[i / kSymCopies];
   for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x) e2[i] = enc[i / copies];
   const uint32_t lane = threadIdx.x & 31;
-  cd.sym = smem + (lane & (kSymCopies - 1)) * 8;
+  cd.sym = smem_addr(smem) + (lane & (kSymCopies - 1)) * 8;
   cd.enc_row = 2 * copies;
   // entry e of copy c is at e2 + (e * copies + c) * 2
-  cd.enc = reinterpret_cast<const unsigned char*>(e2) + (lane & (copies - 1)) * 2;
+  cd.enc = smem_addr(e2) + (lane & (copies - 1)) * 2 - 4096u * cd.enc_row;
   cd.L = L;
 }
 
@@ -86,7 +95,7 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
 // at the segment's first byte; the chunk's symbols are its pieces in order, so the last piece is
 // coded first. Full pieces are 16-byte loads, which a warp's 32 chunks of one group issue as 512
 // consecutive bytes.
-template <int S, bool PAIRS, class Sink>
+template <int S, bool PAIRS, bool CHECK, class Sink>
 __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, const ChunkGeo& g, uint32_t* st,
                                            uint32_t& flags, Sink& sink) {
   int k = (int)g.pieces - 1;
@@ -99,7 +108,7 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
       for (int z = 1; z < S; ++z)
         if (z == q) x = st[z];
       uint32_t w;
-      const uint32_t field = cd.step(src[t], x, w, flags);
+      const uint32_t field = cd.step<CHECK>(src[t], x, w, flags);
 #pragma unroll
       for (int z = 0; z < S; ++z)
         if (z == q) st[z] = x;
@@ -121,14 +130,7 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
              ((uint32_t)src[4 * z + 3] << 24);
     return make_uint4(v[0], v[1], v[2], v[3]);
   };
-  // the next two pieces are always in flight while one is coded (loads are issued 2 pieces ahead)
-  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = make_uint4(0, 0, 0, 0);
-  if (k >= 0) p0 = load_piece(k);
-  if (k >= 1) p1 = load_piece(k - 1);
-  for (; k >= 0; --k) {
-    const uint4 cur = p0;
-    p0 = p1;
-    if (k >= 2) p1 = load_piece(k - 2);
+  auto code_piece = [&](const uint4 cur) {
     const uint32_t wv[4] = {cur.x, cur.y, cur.z, cur.w};
     if (PAIRS) {  // symbols r and r-1: their fields (<= 16 bits each, L <= 256) as one append
 #pragma unroll
@@ -136,8 +138,8 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
         const uint32_t b1 = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
         const uint32_t b2 = __byte_perm(wv[(r - 1) >> 2], 0u, 0x4440u + (uint32_t)((r - 1) & 3));
         uint32_t w1, w2;
-        const uint32_t f1 = cd.step(b1, st[r & (S - 1)], w1, flags);
-        const uint32_t f2 = cd.step(b2, st[(r - 1) & (S - 1)], w2, flags);
+        const uint32_t f1 = cd.step<CHECK>(b1, st[r & (S - 1)], w1, flags);
+        const uint32_t f2 = cd.step<CHECK>(b2, st[(r - 1) & (S - 1)], w2, flags);
         sink(f1 | (f2 << w1), w1 + w2);
       }
     } else {
@@ -145,11 +147,28 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
       for (int r = 15; r >= 0; --r) {
         const uint32_t b = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
         uint32_t w;
-        const uint32_t field = cd.step(b, st[r & (S - 1)], w, flags);
+        const uint32_t field = cd.step<CHECK>(b, st[r & (S - 1)], w, flags);
         sink(field, w);
       }
     }
     sink.piece_done();
+  };
+  // kEncAhead pieces are in flight while one is coded. The piece loop is unrolled by kEncAhead so
+  // that every prefetch slot is a fixed set of registers: a slot is refilled right after it is
+  // consumed, and no register copy ever waits on a load that was issued recently.
+  uint4 pf[kEncAhead];
+#pragma unroll
+  for (int a = 0; a < kEncAhead; ++a) pf[a] = (k >= a) ? load_piece(k - a) : make_uint4(0, 0, 0, 0);
+  while (k >= 0) {
+#pragma unroll
+    for (int a = 0; a < kEncAhead; ++a) {  // slot a holds piece k (the group's a-th)
+      if (k >= 0) {
+        const uint4 cur = pf[a];
+        if (k >= kEncAhead) pf[a] = load_piece(k - kEncAhead);
+        code_piece(cur);
+        --k;
+      }
+    }
   }
 }
 
@@ -162,43 +181,42 @@ struct BitCounter {
 // Write-pass sink: LSB-first bit accumulator; complete words go to a per-thread ring in shared
 // memory, and whole 16-byte-aligned groups of 4 words leave it as one 16-byte store.
 struct RingWriter {
-  uint32_t* ring;     // this thread's row
-  uint32_t* payload;  // stream payload, 16-byte aligned
+  uint32_t ring;         // shared address of this thread's row
+  uint32_t* payload;     // stream payload, 16-byte aligned
   uint32_t wp, fp, end;  // next word to append, next word to store, end of this chunk (payload words)
-  uint32_t a0, a1;    // accumulated bits: a0 holds cnt (< 32) bits, a1 the overflow of the last append
+  uint32_t a0;           // the cnt (< 32) bits not yet in the ring
   uint32_t cnt;
+  __device__ __forceinline__ uint32_t slot(uint32_t word) const { return ring + (word & (kRingWords - 1)) * 4u; }
   // append the low n (<= 32) bits of v; the caller guarantees v < 2^n
   __device__ __forceinline__ void operator()(uint32_t v, uint32_t n) {
     a0 |= v << cnt;
-    a1 |= __funnelshift_l(v, 0u, cnt);  // bits of v beyond position 32 (none when cnt == 0)
+    const uint32_t over = __funnelshift_l(v, 0u, cnt);  // bits of v beyond position 32 (0 when cnt == 0)
     cnt += n;
     if (cnt >= 32) {
-      ring[wp & (kRingWords - 1)] = a0;
+      sts32(slot(wp), a0);
       ++wp;
-      a0 = a1;
-      a1 = 0;
+      a0 = over;
       cnt -= 32;
     }
   }
   __device__ __forceinline__ void piece_done() {
     while ((fp & 3u) != 0 && fp < wp) {  // unaligned head of the chunk
-      if (fp < end) payload[fp] = ring[fp & (kRingWords - 1)];
+      if (fp < end) payload[fp] = lds32(slot(fp));
       ++fp;
     }
     while (fp + 4 <= wp) {
-      if (fp + 4 <= end)
-        *reinterpret_cast<uint4*>(payload + fp) = *reinterpret_cast<const uint4*>(ring + (fp & (kRingWords - 1)));
+      if (fp + 4 <= end) *reinterpret_cast<uint4*>(payload + fp) = lds128(slot(fp));
       fp += 4;
     }
   }
   __device__ __forceinline__ void finish() {
     if (cnt > 0) {
-      ring[wp & (kRingWords - 1)] = a0;
+      sts32(slot(wp), a0);
       ++wp;
     }
     piece_done();
     for (; fp < wp; ++fp)
-      if (fp < end) payload[fp] = ring[fp & (kRingWords - 1)];
+      if (fp < end) payload[fp] = lds32(slot(fp));
   }
 };
 
@@ -222,10 +240,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
   BitCounter bc;
-  code_chunk<S, PAIRS>(cd, in + b.offset[seg], geo, st, flags, bc);
+  code_chunk<S, PAIRS, true>(cd, in + b.offset[seg], geo, st, flags, bc);
   const uint64_t total = (uint64_t)bc.bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
-  if ((flags & 0x80000000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
+  if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
 }
 
 template <int S, bool PAIRS>
@@ -247,18 +265,17 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
   RingWriter rw;
-  rw.ring = reinterpret_cast<uint32_t*>(esm + round_up(enc_table_smem_bytes(lay.R), 16)) + threadIdx.x * kRingStride;
+  rw.ring = smem_addr(esm) + (uint32_t)round_up(enc_table_smem_bytes(lay.R), 16) + threadIdx.x * (kRingStride * 4);
   rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
   rw.wp = rw.fp = (uint32_t)w.word_offset[g];
   rw.end = (uint32_t)w.word_offset[g + 1];
   rw.a0 = 0;
-  rw.a1 = 0;
   rw.cnt = 0;
   uint32_t st[S];
 #pragma unroll
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
-  code_chunk<S, PAIRS>(cd, in + b.offset[seg], geo, st, flags, rw);
+  code_chunk<S, PAIRS, false>(cd, in + b.offset[seg], geo, st, flags, rw);
 #pragma unroll
   for (int q = 0; q < S; ++q) rw(st[q] - cd.L, lay.R);
   rw(1u, 1u);  // sentinel

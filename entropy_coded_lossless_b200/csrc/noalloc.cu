@@ -54,7 +54,6 @@ cudaError_t scratch_address(void** out) {
 
 bool params_ok(const shn_params* p) { return shn_check_params(p) == SHN_OK; }
 
-constexpr int kEncBlockThreads = 128;  // chunks per encoder block (as in shn_encode)
 
 }  // namespace
 

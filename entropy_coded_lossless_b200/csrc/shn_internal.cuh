@@ -62,7 +62,8 @@ __host__ __device__ inline ChunkGeo chunk_geo(uint64_t n, uint32_t C, uint32_t c
 // ---- device table record (include/shn.h: shn_table) -----------------------------------------
 // opaque part: uint2 sym[256] for every raw byte b (u = b ^ 0x80):
 //   .x = bias[s]  (nb = (X + bias) >> 16),
-//   .y = (start[s] + 4096) | (offset << 16) | (w << 24)   with start[s] = cumul_s - f_s,
+//   .y = offset | (w << 8) | (start[s] + 4096) << 16   with start[s] = cumul_s - f_s; bit 15 marks
+//        a byte whose range has no states (absent from the histogram the table was built from),
 // then uint16 enc[L] holding the next state L + slot.
 constexpr uint32_t kOpaqueSymOffset = 0;
 constexpr uint32_t kOpaqueEncOffset = 2048;
@@ -74,6 +75,42 @@ __device__ __forceinline__ const uint2* table_sym(const shn_table* t) {
 }
 __device__ __forceinline__ const uint16_t* table_enc(const shn_table* t) {
   return reinterpret_cast<const uint16_t*>(t->opaque + kOpaqueEncOffset);
+}
+
+// Encoder block size: one thread per chunk, so also the chunks each encoder block codes. The host
+// batching (block_start) and the encoder kernels both use it.
+#ifndef ENC_THREADS
+#define ENC_THREADS 256
+#endif
+constexpr int kEncBlockThreads = ENC_THREADS;
+
+// ---- shared-memory accesses by 32-bit shared-window address ------------------------------------
+// The per-symbol loops address their tables and rings with 32-bit shared addresses (no 64-bit
+// generic-pointer arithmetic). The ring accessors are volatile with a memory clobber so they stay
+// ordered after the cp.async waits and the __syncthreads that publish the data they read.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 // ---- device status word (first 8 bytes of every workspace) -----------------------------------
