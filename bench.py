@@ -44,12 +44,24 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
+    ap.add_argument("--entropy", type=float, default=5.3, choices=[2.0, 4.0, 5.3, 7.9], help="sweep workload")
+    ap.add_argument("--K", type=int, default=None, help="override the workload's range count")
+    ap.add_argument("--log2L", type=int, default=None, help="override the workload's log2 state count")
+    ap.add_argument("--chunk-symbols", type=int, default=None)
+    ap.add_argument("--states", type=int, default=None, help="interleaved states per chunk")
     ap.add_argument("--profile-only", action="store_true",
                     help="run compress + decode twice untimed and exit (the case profiles/ captures)")
     return ap.parse_args()
 
 
-def workload(name, device, seed_offset=0, n_segments=0):
+def apply_overrides(p, args):
+    for key, val in (("K", args.K), ("log2L", args.log2L), ("chunk_symbols", args.chunk_symbols),
+                     ("states_per_chunk", args.states)):
+        if val is not None:
+            p[key] = val
+
+
+def workload(name, device, seed_offset=0, n_segments=0, entropy=5.3):
     """(int8 tensor, segments, params dict, description)."""
     if name == "kv":
         segs = inputs.kv_cache_segments()
@@ -72,9 +84,9 @@ def workload(name, device, seed_offset=0, n_segments=0):
         x, segs, _ = inputs.activation_batch_int8(1024, 65536, seed=3 + seed_offset, device=device)
         desc = "1024 activation tensors x 65536 INT8 (per-tensor tables)"
     else:
-        x = inputs.sweep_stream_int8(5.3, seed=4 + seed_offset, device=device)
+        x = inputs.sweep_stream_int8(entropy, seed=4 + seed_offset, device=device)
         segs = [(0, x.numel())]
-        desc = "1 GiB truncated discrete Laplace, H=5.3 bits"
+        desc = f"1 GiB truncated discrete Laplace, H={entropy} bits"
     return x, segs, dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4), desc
 
 
@@ -98,19 +110,19 @@ def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
 # the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     "decode_kernel": {
-        "bytes_per_symbol": 1.8637,
+        "bytes_per_symbol": 1.8872,
         "source": "decode.cu",
-        "sha256_prefix": "fbee812352b2843e"
+        "sha256_prefix": "2b4d4b18f28e5a01"
     },
     "encode_write_kernel": {
-        "bytes_per_symbol": 1.9429,
+        "bytes_per_symbol": 2.0505,
         "source": "encode.cu",
-        "sha256_prefix": "e69096e9fafd4ba6"
+        "sha256_prefix": "d6fd28e5e1ba08f2"
     },
     "encode_sizes_kernel": {
-        "bytes_per_symbol": 1.0037,
+        "bytes_per_symbol": 1.0036,
         "source": "encode.cu",
-        "sha256_prefix": "e69096e9fafd4ba6"
+        "sha256_prefix": "d6fd28e5e1ba08f2"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0056,
@@ -120,7 +132,7 @@ MEASURED_TRAFFIC = {
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0001,
         "source": "build_tables.cu",
-        "sha256_prefix": "da8b40b8d15eabba"
+        "sha256_prefix": "5ad5c5ee295f0316"
     }
 }
 
@@ -281,7 +293,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    x, segs, p, desc = workload(args.workload, "cpu")
+    x, segs, p, desc = workload(args.workload, "cpu", entropy=args.entropy)
+    apply_overrides(p, args)
     import oracle
 
     cores = oracle.cpu_count()
@@ -341,7 +354,9 @@ def main():
                                              device_id=dev)
     from entropy_coded_lossless_b200 import shn
 
-    x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank, n_segments=args.segments)
+    x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank, n_segments=args.segments,
+                                     entropy=args.entropy)
+    apply_overrides(p_dict, args)
     p = shn.CodecParams(**p_dict)
     codec = shn.Codec(segs, p, device=dev)
     n = codec.n_symbols
@@ -381,6 +396,9 @@ def main():
 
     # events for every timed step, read only after the last one (no host sync inside the region)
     evs_all = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # a workload that fits in L2 is timed with L2 flushed before every step (a 256 MiB write outside
+    # the stage events); its step time is then the sum of the stage events
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if n < (1 << 28) else None
     with ClockSampler(local_rank) as clk:
         for _ in range(args.warmup):
             step()
@@ -392,6 +410,8 @@ def main():
         h0 = time.time()
         t0.record(stream)
         for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
             step(evs_all[i])
         t1.record(stream)
         torch.cuda.synchronize()
@@ -403,7 +423,8 @@ def main():
             stage_ms[k] += evs[i].elapsed_time(evs[i + 1])
     if world > 1:
         torch.distributed.barrier()
-    ms_total = max_over_ranks(t0.elapsed_time(t1), dev)
+    ms_region = t0.elapsed_time(t1) if flush is None else sum(stage_ms.values())
+    ms_total = max_over_ranks(ms_region, dev)
     ms_step = ms_total / args.steps
 
     # correctness of the timed work
@@ -414,38 +435,67 @@ def main():
     stream_np = codec.stream_buf[:nbytes].cpu().numpy()
     rate = stream_rate(stream_np, segs, p_dict, codec.hist.cpu().numpy())
 
-    # e2e through the C ABI with host buffers: pinned H2D of the input, the four calls, D2H of the stream
+    # e2e through the C ABI with host buffers: every step copies its input from pinned host memory,
+    # runs the four calls and copies its stream and status words back. Steps are software-pipelined
+    # over three streams (H2D, compute, D2H; double-buffered device input and stream), so one step's
+    # D2H overlaps the next step's H2D on the other copy engine.
     e2e = None
     if not args.no_e2e:
         h_in = torch.empty(n, dtype=torch.int8, pin_memory=True)
         h_in.copy_(x.cpu())
-        h_out = torch.empty(comp_cap, dtype=torch.uint8, pin_memory=True)
-        h_st = torch.empty(16, dtype=torch.uint8, pin_memory=True)
-        x_e = torch.empty_like(x)
+        h_out = [torch.empty(comp_cap, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        h_st = [torch.empty(16, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        codecs = [codec, shn.Codec(segs, p, device=dev)]
+        outs = [out, torch.empty_like(out)]
+        x_e = [torch.empty_like(x) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        for b in range(2):  # all buffers start free
+            ev_comp[b].record(stream)
+            ev_out[b].record(stream)
 
-        def e2e_step():
-            x_e.copy_(h_in, non_blocking=True)
-            codec.histogram(x_e)
-            codec.build()
-            codec.encode(x_e)
-            codec.decode(codec.stream_buf, comp_cap, out)
-            h_out[:nbytes].copy_(codec.stream_buf[:nbytes], non_blocking=True)
-            h_st[:8].copy_(codec.work_enc[:8], non_blocking=True)
-            h_st[8:16].copy_(codec.work_dec[:8], non_blocking=True)
+        def e2e_step(i):
+            b = i & 1
+            cd = codecs[b]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[b])  # step i-2 no longer reads x_e[b]
+                x_e[b].copy_(h_in, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])  # step i-2's stream has left the device
+            cd.histogram(x_e[b], stream)
+            cd.build(stream)
+            cd.encode(x_e[b], stream)
+            cd.decode(cd.stream_buf, comp_cap, outs[b], stream)
+            ev_comp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                h_out[b][:nbytes].copy_(cd.stream_buf[:nbytes], non_blocking=True)
+                h_st[b][:8].copy_(cd.work_enc[:8], non_blocking=True)
+                h_st[b][8:16].copy_(cd.work_dec[:8], non_blocking=True)
+                ev_out[b].record(s_out)
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ksteps = max(1, min(args.steps, 3))
+        ksteps = max(2, min(args.steps, 6))
         e0.record(stream)
-        for _ in range(ksteps):
-            e2e_step()
+        s_in.wait_event(e0)
+        for i in range(ksteps):
+            e2e_step(i)
+        stream.wait_stream(s_out)
         e1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / ksteps, dev)
+        e2e_ok = all(bool(torch.equal(h_out[b][:nbytes], h_out[0][:nbytes])) for b in range(2)) and \
+            all(int(h_st[b].view(torch.int32)[0]) == 0 and int(h_st[b].view(torch.int32)[2]) == 0 for b in range(2))
         e2e = {"value": whole_job_gbs(n, world, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": n,
-               "d2h_bytes_per_step": nbytes + 16, "ms_per_step": ms_e2e,
-               "what": "pinned H2D input + shn_histogram + shn_build_tables + shn_encode + shn_decode + D2H stream/status"}
+               "d2h_bytes_per_step": nbytes + 16, "ms_per_step": ms_e2e, "correct": e2e_ok,
+               "what": "pinned H2D input + shn_histogram + shn_build_tables + shn_encode + shn_decode + D2H stream/status; "
+                       "steps pipelined over H2D / compute / D2H streams (double-buffered)"}
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
@@ -483,8 +533,8 @@ def main():
             "data": "synthetic",
             "config": {"workload": desc, "K": p.K, "L": 1 << p.log2L, "chunk_symbols": p.chunk_symbols,
                        "states_per_chunk": p.states_per_chunk, "bytes_per_gpu": n,
-                       "l2": "inputs larger than L2 (2 GiB in, ~1.9 GB stream, 2 GiB out per step)"
-                       if n > (1 << 28) else "input smaller than L2; no flush",
+                       "l2": "inputs larger than L2 (input, stream and output each > 126 MB per step)"
+                       if flush is None else "L2 flushed (256 MiB write) before every step; step time = sum of stage events",
                        "parallelism": f"replicas x{world} (independent segments per rank)"},
             "step": "histogram + DP/tables + encode + decode (value = INT8 bytes per step / step time)",
             "stages": stages,

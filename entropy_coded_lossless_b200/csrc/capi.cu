@@ -221,7 +221,6 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
 int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, void* d_work, size_t work_bytes,
                uint8_t* d_out, size_t out_capacity, void* stream) {
   if (!params_ok(p)) return SHN_ERR_INVALID_ARG;
-  if (p->log2L > 8) return SHN_ERR_UNSUPPORTED;
   if (!d_comp || !d_work || (!d_out && out_capacity > 0)) return SHN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(d_comp) & 15) || (reinterpret_cast<uintptr_t>(d_work) & 255))
     return SHN_ERR_INVALID_ARG;

@@ -41,7 +41,10 @@ constexpr int kDecWarps = DEC_WARPS;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr uint32_t kRingQuads = 8;                // 16-byte quads per thread
 constexpr uint32_t kRingBytes = kRingQuads * 16;  // per thread
-constexpr uint32_t kReplicas = 16;
+// Copies of the decode table: 16 (a conflict-free half-warp phase) up to L = 256, then fewer so the
+// replicated table stays at 32 KB: L = 512, 1024, 2048, 4096 keep 8, 4, 2, 1 copies (lanes that share
+// a copy may then conflict on a bank).
+__host__ __device__ inline uint32_t dec_replicas(uint32_t R) { return R <= 8 ? 16u : (16u >> (R - 8)); }
 constexpr uint32_t kStageBytes = 8192;
 
 struct DecHeader {
@@ -147,7 +150,7 @@ struct SmemLayout {
 __host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
   SmemLayout l;
   const uint32_t L = 1u << R;
-  l.table_bytes = L * kReplicas * 8;
+  l.table_bytes = L * dec_replicas(R) * 8;
   l.ring_off = l.table_bytes;
   // table builds happen only while no chunk is being decoded (rings idle, no copies in flight),
   // so the build staging area shares the rings' space
@@ -218,9 +221,10 @@ __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, con
     const uint32_t w = wb[s] & 0xFFu, base = wb[s] >> 8;
     const uint32_t y = nb | (w << 8) | (base << 16) | (((0u - (nb + w)) & 0xFFu) << 24);
     if (replicated) {
-      uint2* row = reinterpret_cast<uint2*>(dsm + i * (kReplicas * 8));
+      const uint32_t reps = dec_replicas(R);
+      uint2* row = reinterpret_cast<uint2*>(dsm + i * (reps * 8));
 #pragma unroll
-      for (uint32_t c = 0; c < kReplicas; ++c) row[c] = make_uint2(dsm_saddr + next * (kReplicas * 8) + c * 8, y);
+      for (uint32_t c = 0; c < reps; ++c) row[c] = make_uint2(dsm_saddr + next * (reps * 8) + c * 8, y);
     } else {
       reinterpret_cast<uint2*>(dsm + t * L * 8)[i] = make_uint2(dsm_saddr + t * L * 8 + next * 8, y);
     }
@@ -277,12 +281,14 @@ struct Fetcher {
       cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
     }
   }
-  // Per 16-symbol piece at most 2 quads (256 bits, the most 16 fields of <= 16 bits can use) leave
-  // the ring, so topping it up with at most 2 fetches keeps it full: no loop, two predicated copies.
-  __device__ __forceinline__ void top_up2(const ChunkCtx& c, int32_t limit) {
+  // Per 16-symbol piece at most N quads leave the ring (2 for fields of <= 16 bits, L <= 256; 3 for
+  // fields of <= 20 bits), so topping it up with at most N fetches keeps it full: no loop, N
+  // predicated copies.
+  template <int N>
+  __device__ __forceinline__ void top_up(const ChunkCtx& c, int32_t limit) {
     const int32_t target = limit > bottom ? limit : bottom;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < N; ++i) {
       if (lo > target) {
         --lo;
         cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
@@ -291,7 +297,9 @@ struct Fetcher {
   }
 };
 
-template <int S, int SH>
+// One chunk. SH = log2 of the table row stride in bytes. PAIRS (fields <= 16 bits, L <= 256): two
+// symbols per window position; otherwise one (fields <= 20 bits).
+template <int S, int SH, bool PAIRS>
 __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
   const uint32_t mask = kRingBytes - 1;
   const uint32_t cb_mod = (uint32_t)(c.cb & mask);
@@ -332,10 +340,28 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
   const uint32_t full = c.pieces - (c.last_len < 16 ? 1u : 0u);
   uint8_t* dst = c.dst;
   for (uint32_t k = 0; k < full; ++k, dst += c.dst_stride) {
-    fe.top_up2(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    fe.top_up<PAIRS ? 2 : 3>(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<1>();
     uint32_t ov[4];
+    if (!PAIRS) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int q = i % S;
+        const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);
+        const uint2 E = lds64(X[q]);
+        const uint32_t r = __funnelshift_l(V, 0u, E.y);
+        const uint32_t Vs = __funnelshift_l(0u, V, E.y);
+        const uint32_t o = __funnelshift_l(Vs, 0u, shr8(E.y));
+        X[q] = E.x + r * (1u << SH);
+        P = add_top_byte(E.y, P);
+        advance();
+        const uint32_t b = add_shr16(E.y, o);
+        // b's low byte into byte i % 4 of the output word (the other bytes are kept)
+        if ((i & 3) == 0) ov[i >> 2] = b;
+        else ov[i >> 2] = __byte_perm(ov[i >> 2], b, (i & 3) == 1 ? 0x3240u : (i & 3) == 2 ? 0x3410u : 0x4210u);
+      }
+    } else {
 #pragma unroll
     for (int pp = 0; pp < 8; ++pp) {
       const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
@@ -345,9 +371,9 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       const uint32_t Va = __funnelshift_l(0u, V, Ea.y);          // V << nb
       const uint32_t wa = shr8(Ea.y);                            // low 5 bits: w
       const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
+      const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
       const uint32_t ba = add_shr16(Ea.y, oa);                   // low byte: base' + offset
       X[qa] = Ea.x + ra * (1u << SH);
-      const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
       P = add_top_byte(Ea.y, P);                                 // P -= nb + w
       const uint2 Eb = lds64(X[qb]);
       const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
@@ -361,6 +387,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
       if ((pp & 1) == 0) ov[pp >> 1] = pair;
       else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
+    }
     }
     if (aligned) {
       *reinterpret_cast<uint4*>(dst) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
@@ -473,8 +500,16 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
         cur_seg = sa;
       }
       if (valid) {
-        c.tbase = dsm_saddr + (lane & (kReplicas - 1)) * 8;
-        if (!decode_chunk<S, 7>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+        c.tbase = dsm_saddr + (lane & (dec_replicas(h.R) - 1)) * 8;
+        bool ok;
+        switch (h.R) {  // row stride: 16 copies x 8 bytes up to L = 256, then 8, 4, 2, 1 copies
+          case 9: ok = decode_chunk<S, 6, false>(c, h.R); break;
+          case 10: ok = decode_chunk<S, 5, false>(c, h.R); break;
+          case 11: ok = decode_chunk<S, 4, false>(c, h.R); break;
+          case 12: ok = decode_chunk<S, 3, false>(c, h.R); break;
+          default: ok = decode_chunk<S, 7, true>(c, h.R); break;
+        }
+        if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
       }
     } else {
       cur_seg = -1;
@@ -484,7 +519,8 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
         build_decode_tables(recs, h, lay, s0, nt, false, dsm, dsm_saddr);
         if (valid && seg >= s0 && seg < s0 + nt) {
           c.tbase = dsm_saddr + (seg - s0) * L * 8;
-          if (!decode_chunk<S, 3>(c, h.R)) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
+          const bool ok = h.R <= 8 ? decode_chunk<S, 3, true>(c, h.R) : decode_chunk<S, 3, false>(c, h.R);
+          if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
         }
       }
     }

@@ -31,13 +31,19 @@ constexpr uint32_t kEncCopyBudget = 16384;        // bytes for the replicated ne
 constexpr uint32_t kRingWords = 16;               // per-thread output staging ring (write pass)
 constexpr uint32_t kRingStride = kRingWords + 4;  // 80-byte rows: 16-byte reads of 8 rows hit distinct banks
 
+#ifndef ENC_SLOT_BYTES
+#define ENC_SLOT_BYTES 4
+#endif
+// Bytes per next-state entry copy: 4 gives every lane its own bank (2 would pack two lanes' copies
+// into one bank word, where lanes 2j and 2j+1 can conflict; measured slower).
+constexpr uint32_t kEncSlot = ENC_SLOT_BYTES;
 __host__ __device__ inline uint32_t enc_copies(uint32_t R) {
   uint32_t c = 32;
-  while (c > 1 && (2u << R) * c > kEncCopyBudget) c >>= 1;
+  while (c > 1 && (kEncSlot << R) * c > kEncCopyBudget) c >>= 1;
   return c;
 }
 __host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t R) {
-  return 256 * kSymCopies * 8 + (2u << R) * enc_copies(R);
+  return 256 * kSymCopies * 8 + (kEncSlot << R) * enc_copies(R);
 }
 
 // Segment of this block: largest s with block_start[s] <= blockIdx.x.
@@ -80,14 +86,15 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   const uint2* sym = table_sym(t);
   const uint16_t* enc = table_enc(t);
   uint2* s2 = reinterpret_cast<uint2*>(smem);
-  uint16_t* e2 = reinterpret_cast<uint16_t*>(smem + 256 * kSymCopies * 8);
+  unsigned char* e2 = smem + 256 * kSymCopies * 8;
   for (uint32_t i = threadIdx.x; i < 256 * kSymCopies; i += blockDim.x) s2[i] = sym[i / kSymCopies];
-  for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x) e2[i] = enc[i / copies];
+  for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x)
+    *reinterpret_cast<uint16_t*>(e2 + i * kEncSlot) = enc[i / copies];
   const uint32_t lane = threadIdx.x & 31;
   cd.sym = smem_addr(smem) + (lane & (kSymCopies - 1)) * 8;
-  cd.enc_row = 2 * copies;
-  // entry e of copy c is at e2 + (e * copies + c) * 2
-  cd.enc = smem_addr(e2) + (lane & (copies - 1)) * 2 - 4096u * cd.enc_row;
+  cd.enc_row = kEncSlot * copies;
+  // entry e of copy c is at e2 + (e * copies + c) * kEncSlot
+  cd.enc = smem_addr(e2) + (lane & (copies - 1)) * kEncSlot - 4096u * cd.enc_row;
   cd.L = L;
 }
 

@@ -156,8 +156,7 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
  *  d_comp      device, comp_bytes of stream, 16-byte aligned.
  *  d_work      device workspace of >= shn_decode_workspace_bytes(p) bytes, 256-byte aligned.
  *  d_out       device, out_capacity bytes, any alignment.
- * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_UNSUPPORTED (log2L > 8 in this build),
- *         SHN_ERR_CUDA; device: SHN_ERR_CORRUPT (bad header/descriptor/index, missing sentinel,
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_CUDA; device: SHN_ERR_CORRUPT (bad header/descriptor/index, missing sentinel,
  *         end-of-chunk state or position check failed), SHN_ERR_CAPACITY (out_capacity too small).
  * A chunk that fails its checks leaves its output bytes unspecified; every other chunk is decoded.
  */

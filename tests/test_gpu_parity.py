@@ -93,6 +93,29 @@ def test_config2_weight_like(orc):
     check_parity(orc, x, [(0, x.size)], shn.CodecParams(16, 7, 4096, 4))
 
 
+def test_config2_plain_tans_l1024(orc):
+    """The comparator of the weight-tensor config: plain tANS (K = 256 identity ranges) at L = 1024,
+    bit-exact on the GPU, and (as on the pages) longer than Shannonic K = 16, L = 128."""
+    x = inputs.weight_like_int8(seed=1).numpy()
+    g_tans, _ = check_parity(orc, x, [(0, x.size)], shn.CodecParams(256, 10, 4096, 4))
+    g_sh = gpu_pipeline(x, [(0, x.size)], shn.CodecParams(16, 7, 4096, 4))
+    pay = lambda g: spec.parse_stream(g["stream"])["segments"][0]["payload_words"]
+    assert pay(g_sh) < pay(g_tans)
+
+
+@pytest.mark.parametrize("K,R,S,C", [(256, 9, 4, 1024), (16, 10, 2, 4096), (200, 11, 8, 256), (256, 12, 1, 128),
+                                     (3, 12, 16, 1024), (32, 9, 4, 65536)])
+def test_large_state_counts(orc, K, R, S, C):
+    """L = 512 ... 4096: fields up to R + 8 bits, one symbol per window position, fewer table copies;
+    ragged segments so tiles straddle segments (plain per-segment tables)."""
+    rng = np.random.default_rng(K + 7 * R)
+    n = 200_003
+    x = inputs.laplace_int8(n, float(rng.choice([3.0, 20.0, 97.0])), seed=K * R).numpy()
+    cuts = sorted(set([0, n] + rng.integers(0, n, 4).tolist()))
+    segs = [(a, b - a) for a, b in zip(cuts[:-1], cuts[1:])]
+    check_parity(orc, x, segs, shn.CodecParams(K, R, C, S))
+
+
 def test_config4_activation_batch_full(orc):
     x, segs, _ = inputs.activation_batch_int8(1024, 65536, seed=3)
     check_parity(orc, x.numpy(), segs, shn.CodecParams(16, 7, 4096, 4), threads=32)
