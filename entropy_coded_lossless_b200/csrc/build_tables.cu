@@ -8,8 +8,10 @@
 // bit for bit, so it uses only integer arithmetic.
 //
 // Work is tiny (O(K·256²/2) min-plus steps per table) and latency-bound; one block of 512 threads
-// per table keeps everything in shared memory: the fixed-point log2 of every range count (a
-// triangular 256x256 table), two DP rows and the K x 257 argmin matrix.
+// per table keeps everything in shared memory: the per-symbol cost factor (w << 24) - LG(count) of
+// every range [j, i) (a triangular 256x256 table of fixed-point log2 values), two DP rows and the
+// K x 257 argmin matrix. The DP layers are split over groups of 4 threads that each own one long and
+// one short end point, so every thread scans about the same number of candidate starts.
 #include "shn_internal.cuh"
 
 namespace shn {
@@ -17,7 +19,6 @@ namespace shn {
 constexpr int kBuildThreads = 512;
 constexpr int kPairs = 256 * 257 / 2;  // ranges [j, i), 0 <= j < i <= 256
 
-__device__ __forceinline__ int pair_index(int j, int i) { return i * (i - 1) / 2 + j; }
 __device__ __forceinline__ uint32_t ceil_log2_width(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
 
 struct BuildShared {
@@ -33,11 +34,71 @@ struct BuildShared {
   long long cost;
 };
 
+// Greedy state allocation on one warp (FORMAT.md §4): every range with a count starts with one
+// state; each further state goes to the range with the largest N_k * (LG(f_k + 1) - LG(f_k)),
+// ties to the smallest k. kPer ranges per lane (K <= 32 * kPer).
+template <int kPer>
+__device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L, int tid) {
+  unsigned long long N[kPer];
+  uint32_t f[kPer];
+  int nonzero = 0;
+  unsigned long long total = 0;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int k = tid + 32 * r;
+    N[r] = (k < K) ? (unsigned long long)(S.pre[S.lo[k + 1]] - S.pre[S.lo[k]]) : 0ull;
+    f[r] = N[r] > 0 ? 1u : 0u;
+    nonzero += (int)f[r];
+    total += N[r];
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    nonzero += __shfl_xor_sync(0xffffffffu, nonzero, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  if (total == 0) {
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) f[r] = (tid == 0 && r == 0) ? L : 0u;
+  } else {
+    // K <= L is checked on the host, so nonzero <= L
+    for (uint32_t step = 0; step < L - (uint32_t)nonzero; ++step) {
+      unsigned long long bg = 0;
+      int bk = 0x7fffffff;
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int k = tid + 32 * r;
+        if (N[r] > 0) {
+          const unsigned long long g = N[r] * (unsigned long long)(S.lgf[f[r] + 1] - S.lgf[f[r]]);
+          if (bk == 0x7fffffff || g > bg || (g == bg && k < bk)) {
+            bg = g;
+            bk = k;
+          }
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long og = __shfl_xor_sync(0xffffffffu, bg, o);
+        const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        if (ok != 0x7fffffff && (bk == 0x7fffffff || og > bg || (og == bg && ok < bk))) {
+          bg = og;
+          bk = ok;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kPer; ++r)
+        if (tid + 32 * r == bk) f[r] += 1;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int k = tid + 32 * r;
+    if (k < K) S.f[k] = f[r];  // S.f[K..255] were zeroed by the caller
+  }
+}
+
 __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsigned long long* __restrict__ hist_all,
                                                                      shn_params p, shn_table* __restrict__ tables_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BuildShared& S = *reinterpret_cast<BuildShared*>(smem_raw);
-  uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));          // kPairs
+  uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));          // kPairs cost factors
   uint8_t* arg = reinterpret_cast<uint8_t*>(lgc + kPairs);                               // K x 257
 
   const int tid = threadIdx.x;
@@ -48,16 +109,30 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   shn_table* out = tables_out + blockIdx.x;
 
   // ---- prefix sums and the 2^32 bound --------------------------------------------------------
-  if (tid == 0) {
-    unsigned long long acc = 0;
-    S.pre[0] = 0;
-    for (int u = 0; u < 256; ++u) {
-      acc += hist[u];
-      S.pre[u + 1] = (uint32_t)acc;
+  if (tid < 32) {  // warp 0: lane l sums counts 8l .. 8l+7, then a shuffle scan over the lanes
+    unsigned long long v[8], acc = 0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = hist[8 * tid + r];  // eight independent loads in flight
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc += v[r];
+    unsigned long long incl = acc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
     }
-    S.status = acc >= (1ull << 32) ? (uint32_t)SHN_ERR_INVALID_ARG : 0u;
-    S.cost = 0;
-    out->n = acc;
+    unsigned long long run = incl - acc;  // exclusive prefix of this lane
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      run += v[r];
+      S.pre[8 * tid + r + 1] = (uint32_t)run;
+    }
+    if (tid == 31) {
+      S.pre[0] = 0;
+      S.status = incl >= (1ull << 32) ? (uint32_t)SHN_ERR_INVALID_ARG : 0u;
+      S.cost = 0;
+      out->n = incl;
+    }
   }
   for (uint32_t f = tid; f <= L; f += kBuildThreads) S.lgf[f] = lg_fixed(f);
   __syncthreads();
@@ -72,14 +147,11 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
 
   // ---- range selection (FORMAT.md §3) ---------------------------------------------------------
   if (K == 256) {
-    if (tid < 256) S.lo[tid] = tid;
-    if (tid == 0) {
-      long long c = 0;
-      for (int u = 0; u < 256; ++u) {
-        const uint32_t n = S.pre[u + 1] - S.pre[u];
-        c -= (long long)n * lg_fixed(n);
-      }
-      S.cost = c;
+    if (tid < 256) {
+      S.lo[tid] = tid;
+      const uint32_t n = S.pre[tid + 1] - S.pre[tid];
+      // two's-complement sum of -n * LG(n) over the 256 singletons (S.cost starts at 0)
+      atomicAdd(reinterpret_cast<unsigned long long*>(&S.cost), 0ull - (unsigned long long)n * lg_fixed(n));
     }
   } else {
     for (int q = tid; q < kPairs; q += kBuildThreads) {
@@ -87,43 +159,64 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
       while (i * (i - 1) / 2 > q) --i;
       while ((i + 1) * i / 2 <= q) ++i;
       const int j = q - i * (i - 1) / 2;
-      lgc[q] = lg_fixed(S.pre[i] - S.pre[j]);
+      // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30
+      lgc[q] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) - (int32_t)lg_fixed(S.pre[i] - S.pre[j]));
     }
     for (int i = tid; i <= 256; i += kBuildThreads) S.drow[0][i] = (i == 0) ? 0 : LLONG_MAX;
     __syncthreads();
-    // two lanes per end point i: lane parity h takes j = jmin + h, jmin + h + 2, ...
-    const int h = tid & 1;
-    const int i = 256 - (tid >> 1);  // 256 .. 1
+    // Balanced min-plus layers: group g of 4 threads owns the end points ia = 256 - g and ib = g + 1
+    // (together ~257 candidate starts whatever g), and its threads take every 4th candidate of the
+    // concatenated lists. Each thread scans its candidates in ascending j with a strict <, and the
+    // group reduction prefers the smaller value, then the smaller j: the smallest j wins ties.
+    const int r4 = tid & 3;
+    const int ia = 256 - (tid >> 2), ib = (tid >> 2) + 1;
     for (int k = 1; k <= K; ++k) {
       const long long* prev = S.drow[(k - 1) & 1];
       long long* cur = S.drow[k & 1];
-      long long best = LLONG_MAX;
-      int bj = 0x7fffffff;
-      if (i >= k) {
-        const int jmax = (k == 1) ? 0 : i - 1;
-        const uint32_t pi = S.pre[i];
-        for (int j = k - 1 + h; j <= jmax; j += 2) {
-          const uint32_t c = pi - S.pre[j];
-          const long long w = (long long)ceil_log2_width((uint32_t)(i - j));
-          const long long cost = (long long)c * (w << 24) - (long long)((unsigned long long)c * lgc[pair_index(j, i)]);
-          const long long v = prev[j] + cost;
-          if (v < best) {
-            best = v;
-            bj = j;
+      const int na = (ia >= k) ? ((k == 1) ? 1 : ia - k + 1) : 0;  // j = k-1 .. (k == 1 ? 0 : i-1)
+      const int nb = (ib >= k) ? ((k == 1) ? 1 : ib - k + 1) : 0;
+      long long best_a = LLONG_MAX, best_b = LLONG_MAX;
+      int bj_a = 0x7fffffff, bj_b = 0x7fffffff;
+      const uint32_t pa = S.pre[ia], pb = S.pre[ib];
+      const int base_a = ia * (ia - 1) / 2, base_b = ib * (ib - 1) / 2;
+      for (int t = r4; t < na + nb; t += 4) {
+        const bool in_a = t < na;
+        const int j = (k - 1) + (in_a ? t : t - na);
+        const uint32_t c = (in_a ? pa : pb) - S.pre[j];
+        const int32_t d = (int32_t)lgc[(in_a ? base_a : base_b) + j];
+        const long long v = prev[j] + (long long)c * (long long)d;  // Cost(j, i-1) = c * (w << 24) - c * LG(c)
+        if (in_a) {
+          if (v < best_a) {
+            best_a = v;
+            bj_a = j;
           }
+        } else if (v < best_b) {
+          best_b = v;
+          bj_b = j;
         }
       }
-      const long long ob = __shfl_xor_sync(0xffffffffu, best, 1);
-      const int oj = __shfl_xor_sync(0xffffffffu, bj, 1);
-      if (ob < best || (ob == best && oj < bj)) {
-        best = ob;
-        bj = oj;
-      }
-      if (h == 0) {
-        if (i >= k) {
-          cur[i] = best;
-          arg[(size_t)(k - 1) * 257 + i] = (uint8_t)bj;
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        const long long oa = __shfl_xor_sync(0xffffffffu, best_a, o);
+        const int oja = __shfl_xor_sync(0xffffffffu, bj_a, o);
+        if (oa < best_a || (oa == best_a && oja < bj_a)) {
+          best_a = oa;
+          bj_a = oja;
         }
+        const long long ob = __shfl_xor_sync(0xffffffffu, best_b, o);
+        const int ojb = __shfl_xor_sync(0xffffffffu, bj_b, o);
+        if (ob < best_b || (ob == best_b && ojb < bj_b)) {
+          best_b = ob;
+          bj_b = ojb;
+        }
+      }
+      if (r4 == 0 && na > 0) {
+        cur[ia] = best_a;
+        arg[(size_t)(k - 1) * 257 + ia] = (uint8_t)bj_a;
+      }
+      if (r4 == 1 && nb > 0) {
+        cur[ib] = best_b;
+        arg[(size_t)(k - 1) * 257 + ib] = (uint8_t)bj_b;
       }
       if (tid == 0) cur[0] = LLONG_MAX;
       if (tid < 257 && tid < k) cur[tid] = LLONG_MAX;
@@ -141,64 +234,15 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   }
   __syncthreads();
   if (tid == 0) S.lo[K] = 256;
+  if (tid < 256) S.f[tid] = 0;
   __syncthreads();
 
   // ---- state counts (FORMAT.md §4): one warp, greedy with smallest-k tie-break ---------------
   if (tid < 32) {
-    constexpr int kPer = 8;  // ranges per lane (K <= 256)
-    unsigned long long N[kPer];
-    uint32_t f[kPer];
-    int nonzero = 0;
-    unsigned long long total = 0;
-#pragma unroll
-    for (int r = 0; r < kPer; ++r) {
-      const int k = tid + 32 * r;
-      N[r] = (k < K) ? (unsigned long long)(S.pre[S.lo[k + 1]] - S.pre[S.lo[k]]) : 0ull;
-      f[r] = N[r] > 0 ? 1u : 0u;
-      nonzero += (int)f[r];
-      total += N[r];
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      nonzero += __shfl_xor_sync(0xffffffffu, nonzero, o);
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-    }
-    if (total == 0) {
-#pragma unroll
-      for (int r = 0; r < kPer; ++r) f[r] = (tid == 0 && r == 0) ? L : 0u;
-    } else {
-      // K <= L is checked on the host, so nonzero <= L
-      for (uint32_t step = 0; step < L - (uint32_t)nonzero; ++step) {
-        unsigned long long bg = 0;
-        int bk = 0x7fffffff;
-#pragma unroll
-        for (int r = 0; r < kPer; ++r) {
-          const int k = tid + 32 * r;
-          if (N[r] > 0) {
-            const unsigned long long g = N[r] * (unsigned long long)(S.lgf[f[r] + 1] - S.lgf[f[r]]);
-            if (bk == 0x7fffffff || g > bg || (g == bg && k < bk)) {
-              bg = g;
-              bk = k;
-            }
-          }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          const unsigned long long og = __shfl_xor_sync(0xffffffffu, bg, o);
-          const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
-          if (ok != 0x7fffffff && (bk == 0x7fffffff || og > bg || (og == bg && ok < bk))) {
-            bg = og;
-            bk = ok;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kPer; ++r)
-          if (tid + 32 * r == bk) f[r] += 1;
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kPer; ++r) {
-      const int k = tid + 32 * r;
-      if (k < 256) S.f[k] = (k < K) ? f[r] : 0u;
-    }
+    if (K <= 32) normalize_warp<1>(S, K, L, tid);
+    else if (K <= 64) normalize_warp<2>(S, K, L, tid);
+    else if (K <= 128) normalize_warp<4>(S, K, L, tid);
+    else normalize_warp<8>(S, K, L, tid);
   }
   __syncthreads();
   if (tid == 0) {

@@ -42,12 +42,15 @@ int sm_count() {
   return n;
 }
 
+// Encode workspace: status word, per-chunk word counts, their exclusive prefix, scan block sums
+// (`total`, enough for the two-pass encoder); then, for the single-pass encoder, one worst-case
+// slot per chunk (`total_slots`).
 struct EncWorkLayout {
-  size_t status_off, words_off, offsets_off, sums_off, total;
-  uint32_t scan_blocks;
+  size_t status_off, words_off, offsets_off, sums_off, total, slots_off, total_slots;
+  uint32_t scan_blocks, slot_words;
 };
 
-EncWorkLayout enc_work_layout(uint64_t total_chunks) {
+EncWorkLayout enc_work_layout(uint64_t total_chunks, const shn_params* p) {
   EncWorkLayout l;
   l.scan_blocks = (uint32_t)((total_chunks + kScanBlock - 1) / kScanBlock);
   l.status_off = 0;
@@ -55,6 +58,9 @@ EncWorkLayout enc_work_layout(uint64_t total_chunks) {
   l.offsets_off = l.words_off + round_up(4ull * total_chunks, 256);
   l.sums_off = l.offsets_off + round_up(8ull * (total_chunks + 1), 256);
   l.total = l.sums_off + round_up(8ull * (l.scan_blocks + 1), 256);
+  l.slot_words = (uint32_t)round_up(chunk_max_words(p->states_per_chunk, p->log2L, p->chunk_symbols), 4);
+  l.slots_off = l.total;
+  l.total_slots = l.slots_off + round_up(4ull * l.slot_words * total_chunks, 256);
   return l;
 }
 
@@ -94,7 +100,13 @@ size_t shn_encode_bound(const shn_params* p, const shn_segment* h_segs, uint32_t
 size_t shn_encode_workspace_bytes(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs) {
   uint64_t tc = 0;
   if (!params_ok(p) || !segs_ok(h_segs, n_segs, &tc, nullptr, p->chunk_symbols)) return 0;
-  return enc_work_layout(tc).total;
+  return enc_work_layout(tc, p).total_slots;
+}
+
+size_t shn_encode_workspace_bytes_min(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs) {
+  uint64_t tc = 0;
+  if (!params_ok(p) || !segs_ok(h_segs, n_segs, &tc, nullptr, p->chunk_symbols)) return 0;
+  return enc_work_layout(tc, p).total;
 }
 
 size_t shn_decode_workspace_bytes(const shn_params* p) { return params_ok(p) ? 256 : 0; }
@@ -150,8 +162,9 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
     return SHN_ERR_INVALID_ARG;
   // word offsets inside the payload are 32-bit: streams are limited to 16 GiB
   if (shn_encode_bound(p, h_segs, n_segs) > (16ull << 30)) return SHN_ERR_INVALID_ARG;
-  const EncWorkLayout wl = enc_work_layout(tc);
+  const EncWorkLayout wl = enc_work_layout(tc, p);
   if (work_bytes < wl.total) return SHN_ERR_WORKSPACE;
+  const bool single_pass = work_bytes >= wl.total_slots;
   EncodeLayout lay;
   lay.n_segs = n_segs;
   lay.K = p->K;
@@ -172,6 +185,8 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
   w.word_offset = reinterpret_cast<unsigned long long*>(wb + wl.offsets_off);
   w.block_sums = reinterpret_cast<unsigned long long*>(wb + wl.sums_off);
   w.scan_blocks = wl.scan_blocks;
+  w.slots = single_pass ? reinterpret_cast<uint32_t*>(wb + wl.slots_off) : nullptr;
+  w.slot_words = single_pass ? wl.slot_words : 0u;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const shn_table* tables = static_cast<const shn_table*>(d_tables);
   if (cudaMemsetAsync(wb, 0, 8, s) != cudaSuccess) return SHN_ERR_CUDA;
@@ -202,8 +217,12 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
       b.total_blocks = (uint32_t)blocks;
     }
   }
-  for (const EncBatch& b : batches)
-    if (launch_encode_sizes(d_in, b, tables, lay, w, 0, s) != cudaSuccess) return SHN_ERR_CUDA;
+  // single pass: code every chunk into its slot (recording sizes); two passes: count sizes first
+  for (const EncBatch& b : batches) {
+    const cudaError_t e = single_pass ? launch_encode_write(d_in, b, tables, lay, w, d_out, true, s)
+                                      : launch_encode_sizes(d_in, b, tables, lay, w, 0, s);
+    if (e != cudaSuccess) return SHN_ERR_CUDA;
+  }
   if (launch_scan(w, tc, s) != cudaSuccess) return SHN_ERR_CUDA;
   bool first = true;
   for (const EncBatch& b : batches) {
@@ -213,8 +232,12 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
   if (n_segs == 0) {
     if (launch_encode_empty(lay, w, d_out, d_out_bytes, s) != cudaSuccess) return SHN_ERR_CUDA;
   }
-  for (const EncBatch& b : batches)
-    if (launch_encode_write(d_in, b, tables, lay, w, d_out, 0, s) != cudaSuccess) return SHN_ERR_CUDA;
+  if (single_pass) {
+    if (launch_encode_compact(lay, w, d_out, sm_count(), s) != cudaSuccess) return SHN_ERR_CUDA;
+  } else {
+    for (const EncBatch& b : batches)
+      if (launch_encode_write(d_in, b, tables, lay, w, d_out, false, s) != cudaSuccess) return SHN_ERR_CUDA;
+  }
   return SHN_OK;
 }
 

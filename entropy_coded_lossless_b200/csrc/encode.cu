@@ -253,7 +253,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t
   if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
 }
 
-template <int S, bool PAIRS>
+// Writes every chunk's words. Two-pass mode (SLOTS = false): at the chunk's final place in the
+// stream, from the word offsets of the scan. Single-pass mode (SLOTS = true): into the chunk's own
+// worst-case-size slot in the workspace, recording the word count (and, as the size pass would,
+// flagging symbols absent from the table); encode_compact_kernel then moves the slots into place.
+template <int S, bool PAIRS, bool SLOTS>
 __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t* __restrict__ in,
                                                                    const __grid_constant__ EncBatch b,
                                                                    const shn_table* __restrict__ tables,
@@ -273,20 +277,55 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
   RingWriter rw;
   rw.ring = smem_addr(esm) + (uint32_t)round_up(enc_table_smem_bytes(lay.R), 16) + threadIdx.x * (kRingStride * 4);
-  rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
-  rw.wp = rw.fp = (uint32_t)w.word_offset[g];
-  rw.end = (uint32_t)w.word_offset[g + 1];
+  if (SLOTS) {
+    rw.payload = w.slots + g * w.slot_words;
+    rw.wp = rw.fp = 0;
+    rw.end = w.slot_words;
+  } else {
+    rw.payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
+    rw.wp = rw.fp = (uint32_t)w.word_offset[g];
+    rw.end = (uint32_t)w.word_offset[g + 1];
+  }
   rw.a0 = 0;
   rw.cnt = 0;
   uint32_t st[S];
 #pragma unroll
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
-  code_chunk<S, PAIRS, false>(cd, in + b.offset[seg], geo, st, flags, rw);
+  code_chunk<S, PAIRS, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
 #pragma unroll
   for (int q = 0; q < S; ++q) rw(st[q] - cd.L, lay.R);
   rw(1u, 1u);  // sentinel
   rw.finish();
+  if (SLOTS) {
+    w.chunk_words[g] = rw.wp;
+    if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, (uint32_t)g);
+  }
+}
+
+// Single-pass mode: one warp per chunk copies its words from the slot to the final place (32
+// consecutive words per step, four steps in flight per lane).
+__global__ void __launch_bounds__(256) encode_compact_kernel(const EncodeLayout lay, EncodeWork w,
+                                                             uint8_t* __restrict__ out) {
+  if (*(volatile uint32_t*)&w.status->status != 0) return;
+  uint32_t* payload = reinterpret_cast<uint32_t*>(out + lay.payload_offset);
+  const uint32_t lane = threadIdx.x & 31;
+  const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
+  for (uint64_t g = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < lay.total_chunks; g += warps) {
+    const uint32_t* __restrict__ src = w.slots + g * w.slot_words;
+    uint32_t* __restrict__ dst = payload + w.word_offset[g];
+    const uint32_t n = w.chunk_words[g];
+    uint32_t i = lane;
+    for (; i + 96 < n; i += 128) {
+      const uint32_t v0 = __ldcs(src + i), v1 = __ldcs(src + i + 32), v2 = __ldcs(src + i + 64),
+                     v3 = __ldcs(src + i + 96);
+      dst[i] = v0;
+      dst[i + 32] = v1;
+      dst[i + 64] = v2;
+      dst[i + 96] = v3;
+    }
+    for (; i < n; i += 32) dst[i] = __ldcs(src + i);
+  }
 }
 
 // ---- exclusive scan of the chunk word counts (3 small kernels, no inter-block waits) ----------
@@ -457,14 +496,14 @@ static cudaError_t launch_sizes_t(const uint8_t* d_in, const EncBatch& b, const 
   encode_sizes_kernel<S, PAIRS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w);
   return cudaGetLastError();
 }
-template <int S, bool PAIRS>
+template <int S, bool PAIRS, bool SLOTS>
 static cudaError_t launch_write_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
   const size_t smem = round_up(enc_table_smem_bytes(lay.R), 16) + kEncThreads * kRingStride * 4;
-  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, PAIRS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, PAIRS, SLOTS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  encode_write_kernel<S, PAIRS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
+  encode_write_kernel<S, PAIRS, SLOTS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
   return cudaGetLastError();
 }
 
@@ -476,9 +515,12 @@ static cudaError_t sizes_dispatch(const uint8_t* d_in, const EncBatch& b, const 
 }
 template <int S>
 static cudaError_t write_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
-                                  const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
-  return lay.R <= 8 ? launch_write_t<S, true>(d_in, b, t, lay, w, d_out, s)
-                    : launch_write_t<S, false>(d_in, b, t, lay, w, d_out, s);
+                                  const EncodeWork& w, uint8_t* d_out, bool slots, cudaStream_t s) {
+  if (slots)
+    return lay.R <= 8 ? launch_write_t<S, true, true>(d_in, b, t, lay, w, d_out, s)
+                      : launch_write_t<S, false, true>(d_in, b, t, lay, w, d_out, s);
+  return lay.R <= 8 ? launch_write_t<S, true, false>(d_in, b, t, lay, w, d_out, s)
+                    : launch_write_t<S, false, false>(d_in, b, t, lay, w, d_out, s);
 }
 
 cudaError_t launch_encode_sizes(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
@@ -495,17 +537,26 @@ cudaError_t launch_encode_sizes(const uint8_t* d_in, const EncBatch& b, const sh
 }
 
 cudaError_t launch_encode_write(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
-                                const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, int,
+                                const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, bool slots,
                                 cudaStream_t s) {
   if (b.total_blocks == 0) return cudaSuccess;
   switch (lay.S) {
-    case 1: return write_dispatch<1>(d_in, b, d_tables, lay, w, d_out, s);
-    case 2: return write_dispatch<2>(d_in, b, d_tables, lay, w, d_out, s);
-    case 4: return write_dispatch<4>(d_in, b, d_tables, lay, w, d_out, s);
-    case 8: return write_dispatch<8>(d_in, b, d_tables, lay, w, d_out, s);
-    case 16: return write_dispatch<16>(d_in, b, d_tables, lay, w, d_out, s);
+    case 1: return write_dispatch<1>(d_in, b, d_tables, lay, w, d_out, slots, s);
+    case 2: return write_dispatch<2>(d_in, b, d_tables, lay, w, d_out, slots, s);
+    case 4: return write_dispatch<4>(d_in, b, d_tables, lay, w, d_out, slots, s);
+    case 8: return write_dispatch<8>(d_in, b, d_tables, lay, w, d_out, slots, s);
+    case 16: return write_dispatch<16>(d_in, b, d_tables, lay, w, d_out, slots, s);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_encode_compact(const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, int sm_count,
+                                  cudaStream_t s) {
+  if (lay.total_chunks == 0) return cudaSuccess;
+  const uint64_t want = (lay.total_chunks + 7) / 8;  // 8 warps per block, one chunk per warp
+  const uint64_t cap = (uint64_t)sm_count * 8;
+  encode_compact_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(lay, w, d_out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_scan(const EncodeWork& w, uint64_t total_chunks, cudaStream_t s) {

@@ -99,6 +99,8 @@ int shn_encode_static(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n
   w.word_offset = reinterpret_cast<unsigned long long*>(sb + kWordsBytes);
   w.block_sums = reinterpret_cast<unsigned long long*>(sb + kWordsBytes + kOffsetsBytes);
   w.scan_blocks = (uint32_t)((tc + kScanBlock - 1) / kScanBlock);
+  w.slots = nullptr;  // the two-pass encoder: no per-chunk slots
+  w.slot_words = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const shn_table* tables = static_cast<const shn_table*>(d_tables);
   // Only the status must start at zero: every scratch word the passes read is written first
@@ -134,7 +136,7 @@ int shn_encode_static(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n
       cudaError_t e = cudaSuccess;
       if (pass == 0) e = launch_encode_sizes(d_in, b, tables, lay, w, 0, s);
       if (pass == 1) e = launch_encode_header(b, tables, lay, w, d_out, d_out_bytes, first, s);
-      if (pass == 2) e = launch_encode_write(d_in, b, tables, lay, w, d_out, 0, s);
+      if (pass == 2) e = launch_encode_write(d_in, b, tables, lay, w, d_out, false, s);
       if (e != cudaSuccess) return SHN_ERR_CUDA;
       first = false;
     }

@@ -127,14 +127,15 @@ __device__ __forceinline__ void report(DeviceStatus* st, uint32_t code, uint32_t
 __device__ __forceinline__ uint32_t lg_fixed(uint32_t n) {
   if (n == 0) return 0;
   const int e = 31 - __clz(n);
-  unsigned long long m = (unsigned long long)n << (31 - e);
+  uint32_t m = n << (31 - e);  // mantissa in Q1.31: [2^31, 2^32)
   uint32_t frac = 0;
 #pragma unroll
   for (int it = 0; it < 24; ++it) {
-    m = (m * m) >> 31;
-    const uint32_t bit = (uint32_t)(m >> 32);  // 1 iff m >= 2^32 (m < 2^33)
+    // square, keep 31 fraction bits: p = m*m >> 31 (33 bits); the next bit is p >= 2, then halve
+    const uint32_t hi = __umulhi(m, m), lo = m * m;
+    const uint32_t bit = hi >> 31;
+    m = bit ? hi : __funnelshift_l(lo, hi, 1);
     frac = (frac << 1) | bit;
-    m >>= bit;
   }
   return ((uint32_t)e << 24) | frac;
 }
@@ -187,6 +188,8 @@ struct EncodeWork {
   unsigned long long* word_offset;  // exclusive prefix over all chunks, total at [total_chunks]
   unsigned long long* block_sums;
   uint32_t scan_blocks;
+  uint32_t* slots;       // single-pass mode: chunk g's words at slots + g * slot_words (else null)
+  uint32_t slot_words;   // worst-case words per chunk, a multiple of 4
 };
 constexpr uint32_t kScanBlock = 1024;  // chunks reduced per scan block
 
@@ -199,8 +202,10 @@ cudaError_t launch_encode_header(const EncBatch& b, const shn_table* d_tables, c
 cudaError_t launch_encode_empty(const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, uint64_t* d_out_bytes,
                                 cudaStream_t s);
 cudaError_t launch_encode_write(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
-                                const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, int threads,
+                                const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, bool slots,
                                 cudaStream_t s);
+cudaError_t launch_encode_compact(const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, int sm_count,
+                                  cudaStream_t s);
 
 cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
                           uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s);

@@ -28,7 +28,7 @@ TABLE_PUBLIC_BYTES = 800
 
 EXPORTED = [
     "shn_version", "shn_status_string", "shn_check_params", "shn_table_bytes", "shn_encode_bound",
-    "shn_encode_workspace_bytes", "shn_decode_workspace_bytes", "shn_histogram", "shn_build_tables",
+    "shn_encode_workspace_bytes", "shn_encode_workspace_bytes_min", "shn_decode_workspace_bytes", "shn_histogram", "shn_build_tables",
     "shn_encode", "shn_decode", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
 ]
 
@@ -78,6 +78,7 @@ def lib():
             "shn_table_bytes": (sz, [P]),
             "shn_encode_bound": (sz, [P, vp, u32]),
             "shn_encode_workspace_bytes": (sz, [P, vp, u32]),
+            "shn_encode_workspace_bytes_min": (sz, [P, vp, u32]),
             "shn_decode_workspace_bytes": (sz, [P]),
             "shn_histogram": (i32, [vp, vp, u32, vp, vp]),
             "shn_build_tables": (i32, [vp, u32, P, vp, vp]),
@@ -154,7 +155,13 @@ def encode_bound(p: CodecParams, segments) -> int:
 
 
 def encode_workspace_bytes(p: CodecParams, segments) -> int:
+    """Workspace for the single-pass encoder (one worst-case slot per chunk)."""
     return int(lib().shn_encode_workspace_bytes(ctypes.byref(p.c()), _segments(segments), len(segments)))
+
+
+def encode_workspace_bytes_min(p: CodecParams, segments) -> int:
+    """Smallest encoder workspace (two-pass mode)."""
+    return int(lib().shn_encode_workspace_bytes_min(ctypes.byref(p.c()), _segments(segments), len(segments)))
 
 
 def decode_workspace_bytes(p: CodecParams) -> int:
@@ -227,14 +234,17 @@ def empty_aligned(nbytes: int, device, align: int = 256) -> torch.Tensor:
 class Codec:
     """Holds the device buffers for repeated encode/decode of one segment layout."""
 
-    def __init__(self, segments, p: CodecParams = CodecParams(), device="cuda"):
+    def __init__(self, segments, p: CodecParams = CodecParams(), device="cuda", single_pass=True):
+        """single_pass: allocate the encoder workspace that lets every chunk be coded once into its
+        own slot (about the stream bound); otherwise the minimal one (two-pass encoder)."""
         self.p = p
         self.segments = [(int(o), int(n)) for o, n in segments]
         self.device = torch.device(device)
         ns = len(self.segments)
         self.hist = torch.zeros(max(1, ns) * 256, dtype=torch.int64, device=self.device)
         self.tables = empty_aligned(max(1, ns) * TABLE_BYTES, self.device)
-        self.work_enc = empty_aligned(encode_workspace_bytes(p, self.segments), self.device)
+        wsize = encode_workspace_bytes if single_pass else encode_workspace_bytes_min
+        self.work_enc = empty_aligned(wsize(p, self.segments), self.device)
         self.work_dec = empty_aligned(decode_workspace_bytes(p), self.device)
         self.bound = encode_bound(p, self.segments)
         if self.bound == 0:

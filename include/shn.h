@@ -92,8 +92,16 @@ size_t shn_table_bytes(const shn_params* p);
 /* Largest SHN1 stream shn_encode can produce for these segments (0 on bad arguments). */
 size_t shn_encode_bound(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs);
 
-/* Device workspace shn_encode needs (per-chunk sizes and scan scratch + the status word). */
+/* Device workspace for shn_encode's single-pass mode: the status word, per-chunk sizes and scan
+ * scratch, plus one worst-case slot per chunk (about shn_encode_bound bytes in all). With this much
+ * workspace every chunk's state machine runs once and a copy pass moves the slots into place. */
 size_t shn_encode_workspace_bytes(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs);
+
+/* The smallest workspace shn_encode accepts (status word, per-chunk sizes and scan scratch, a few
+ * bytes per chunk). Below shn_encode_workspace_bytes it runs in two passes: one to size every chunk,
+ * one to write it at its final place (the state machine runs twice). No counterpart in the paper:
+ * a memory/time trade of this GPU implementation. */
+size_t shn_encode_workspace_bytes_min(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs);
 
 /* Device workspace shn_decode needs (the status word only). */
 size_t shn_decode_workspace_bytes(const shn_params* p);
@@ -134,8 +142,9 @@ int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params
  *                16-byte aligned (SHN_ERR_INVALID_ARG otherwise).
  *  h_segs        host, n_segs segments; segment s is coded with table s of d_tables.
  *  d_tables      device, n_segs records from shn_build_tables with the same params.
- *  d_work        device workspace of >= shn_encode_workspace_bytes(p, h_segs, n_segs) bytes,
- *                256-byte aligned. Its first 8 bytes receive the device status.
+ *  d_work        device workspace of >= shn_encode_workspace_bytes_min(p, h_segs, n_segs) bytes,
+ *                256-byte aligned; >= shn_encode_workspace_bytes(...) selects the single-pass
+ *                mode (same output). Its first 8 bytes receive the device status.
  *  d_out         device, out_capacity bytes, 16-byte aligned; receives the stream.
  *  d_out_bytes   device uint64: the stream size in bytes (written even when it exceeds the
  *                capacity, in which case the device status is SHN_ERR_CAPACITY and d_out holds

@@ -54,7 +54,12 @@ def test_encode_bound_matches_format(lib, orc, K, R, S, C):
     segs = [(0, 65536), (65536, 0), (65536, 12345), (77881, 1)]
     p = shn.CodecParams(K, R, C, S)
     assert shn.encode_bound(p, segs) == orc.stream_bound(K, R, S, C, segs)
-    assert shn.encode_workspace_bytes(p, segs) >= 256
+    wmin, wfull = shn.encode_workspace_bytes_min(p, segs), shn.encode_workspace_bytes(p, segs)
+    assert 256 <= wmin < wfull
+    # the single-pass slots hold every chunk at its worst case: the bound's payload, give or take
+    # the rounding of each slot to 4 words and of each region to 256 bytes
+    payload_bound = orc.stream_bound(K, R, S, C, segs) - orc.stream_bound(K, R, S, C, [])
+    assert wfull - wmin >= payload_bound - 16 * len(segs) - 4096
     assert shn.decode_workspace_bytes(p) == 256
 
 

@@ -24,10 +24,10 @@ def _lib():
     shn.lib()
 
 
-def gpu_pipeline(x_cpu, segs, p: shn.CodecParams):
+def gpu_pipeline(x_cpu, segs, p: shn.CodecParams, single_pass=True):
     """histogram → tables → encode → decode on the device; returns host copies."""
     x = x_cpu.to(DEV) if isinstance(x_cpu, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(x_cpu)).to(DEV)
-    codec = shn.Codec(segs, p)
+    codec = shn.Codec(segs, p, single_pass=single_pass)
     codec.compress(x)
     st, det = codec.status("enc")
     assert st == 0, (st, det)
@@ -42,8 +42,8 @@ def gpu_pipeline(x_cpu, segs, p: shn.CodecParams):
     return dict(stream=stream.cpu().numpy(), out=out.cpu().numpy(), hist=hist, tables=tables, codec=codec)
 
 
-def check_parity(orc, x_np, segs, p: shn.CodecParams, threads=8):
-    g = gpu_pipeline(x_np, segs, p)
+def check_parity(orc, x_np, segs, p: shn.CodecParams, threads=8, single_pass=True):
+    g = gpu_pipeline(x_np, segs, p, single_pass)
     xb = np.ascontiguousarray(x_np).view(np.uint8).reshape(-1)
     # histograms
     for i, (o, n) in enumerate(segs):
@@ -271,11 +271,26 @@ def test_decoder_reports_corruption(orc):
     assert detected >= 10
 
 
-def test_encoder_reports_capacity():
+@pytest.mark.parametrize("K,R,S,C", [(16, 7, 4, 4096), (5, 10, 2, 1024), (64, 8, 16, 384)])
+def test_two_pass_mode(orc, K, R, S, C):
+    """With the minimal workspace the encoder sizes every chunk first and writes it in place; the
+    stream is the same bytes as the oracle's (and the single-pass mode's)."""
+    rng = np.random.default_rng(K * R)
+    n = 250_001
+    x = inputs.laplace_int8(n, float(rng.choice([2.0, 9.0, 60.0])), seed=R).numpy()
+    cuts = sorted(set([0, n] + rng.integers(0, n, 3).tolist()))
+    segs = [(a, b - a) for a, b in zip(cuts[:-1], cuts[1:])]
+    p = shn.CodecParams(K, R, C, S)
+    assert shn.encode_workspace_bytes_min(p, segs) < shn.encode_workspace_bytes(p, segs)
+    check_parity(orc, x, segs, p, single_pass=False)
+
+
+@pytest.mark.parametrize("single_pass", [True, False])
+def test_encoder_reports_capacity(single_pass):
     p = shn.CodecParams(16, 7, 4096, 4)
     x = inputs.laplace_int8(100_000, 7.0, seed=2).to(DEV)
     segs = [(0, x.numel())]
-    codec = shn.Codec(segs, p)
+    codec = shn.Codec(segs, p, single_pass=single_pass)
     codec.histogram(x)
     codec.build()
     small = shn.empty_aligned(20_000, DEV, 16)
@@ -287,12 +302,13 @@ def test_encoder_reports_capacity():
         shn.shn_encode(x, segs, codec.tables, p, codec.work_enc, small[:10], codec.out_bytes)
 
 
-def test_encoder_rejects_foreign_table():
+@pytest.mark.parametrize("single_pass", [True, False])
+def test_encoder_rejects_foreign_table(single_pass):
     # a table built for a one-value segment cannot code other symbols: device status, no fault
     p = shn.CodecParams(16, 7, 4096, 4)
     a = torch.full((8192,), 3, dtype=torch.int8, device=DEV)
     b = inputs.laplace_int8(8192, 7.0, seed=3).to(DEV)
-    codec = shn.Codec([(0, 8192)], p)
+    codec = shn.Codec([(0, 8192)], p, single_pass=single_pass)
     codec.histogram(a)
     codec.build()
     codec.encode(b)
