@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused decode+dequantise measurement (kv)")
     ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
     ap.add_argument("--entropy", type=float, default=5.3, choices=[2.0, 4.0, 5.3, 7.9], help="sweep workload")
     ap.add_argument("--K", type=int, default=None, help="override the workload's range count")
@@ -497,8 +498,50 @@ def main():
                "what": "pinned H2D input + shn_histogram + shn_build_tables + shn_encode + shn_decode + D2H stream/status; "
                        "steps pipelined over H2D / compute / D2H streams (double-buffered)"}
 
+    # Decode fused with the KV cache's dequantisation (bf16 = int8 x scale per head_dim group of 128),
+    # against the unfused path a user would otherwise run: shn_decode, then a PyTorch dequantisation.
+    fused = None
+    if args.workload == "kv" and not args.segments and not args.no_fused:
+        scales = inputs.kv_cache_scales(seed=2 + rank, device=dev)
+        y16 = torch.empty(n, dtype=torch.bfloat16, device=dev)
+
+        def run_fused():
+            shn.shn_decode_bf16(codec.stream_buf, comp_cap, p, scales, 7, codec.work_dec, y16)
+
+        def run_unfused():
+            codec.decode(codec.stream_buf, comp_cap, out)
+            return (out.view(torch.int8).view(-1, 128).float() * scales[:, None]).to(torch.bfloat16).reshape(-1)
+
+        def timed(fn, reps=5):
+            fn()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                r = fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            return sorted(ts)[len(ts) // 2], r
+
+        ms_f, _ = timed(run_fused)
+        fused_ok = codec.status("dec")[0] == 0
+        ms_u, y_ref = timed(run_unfused)
+        fused_ok = fused_ok and torch.equal(y16.view(torch.int16), y_ref.view(torch.int16))
+        del y_ref
+        torch.cuda.empty_cache()
+        fused = {"what": "shn_decode_bf16: decode + bf16 dequantisation (scale per 128 values) in one kernel",
+                 "ms": ms_f, "gbs_int8": n / (ms_f * 1e-3) / 1e9,
+                 "alg_bytes_per_launch": nbytes + 2 * n + 4 * (n >> 7),
+                 "unfused_ms": ms_u, "unfused": "shn_decode then (int8.float() * scale).to(bfloat16) in PyTorch",
+                 "speedup_vs_unfused": ms_u / ms_f, "matches_unfused": bool(fused_ok)}
+
     if rank == 0:
         peak, peak_kind = measured_peaks()
+        if fused is not None:
+            fused["achieved_gbs"] = fused["alg_bytes_per_launch"] / (fused["ms"] * 1e-3) / 1e9
+            fused["frac"] = fused["achieved_gbs"] / peak
         stages = {}
         for k, v in stage_ms.items():
             ms = v / args.steps
@@ -545,6 +588,7 @@ def main():
             "stream_bytes": nbytes,
             "correct": bool(ok),
             "clocks": clk.summary(),
+            "decode_bf16_fused": fused,
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
         }

@@ -257,6 +257,26 @@ int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, vo
   return SHN_OK;
 }
 
+int shn_decode_bf16(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, const float* d_scales,
+                    size_t n_scales, uint32_t log2_group, void* d_work, size_t work_bytes, uint16_t* d_out,
+                    size_t out_elems, void* stream) {
+  if (!params_ok(p)) return SHN_ERR_INVALID_ARG;
+  if (!d_comp || !d_work || !d_scales || (!d_out && out_elems > 0)) return SHN_ERR_INVALID_ARG;
+  if (log2_group < 4 || log2_group > 31) return SHN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_comp) & 15) || (reinterpret_cast<uintptr_t>(d_work) & 255) ||
+      (reinterpret_cast<uintptr_t>(d_out) & 15) || (reinterpret_cast<uintptr_t>(d_scales) & 3))
+    return SHN_ERR_INVALID_ARG;
+  if (work_bytes < 256) return SHN_ERR_WORKSPACE;
+  if (comp_bytes < kHeaderBytes) return SHN_ERR_CORRUPT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceStatus* st = static_cast<DeviceStatus*>(d_work);
+  if (cudaMemsetAsync(st, 0, sizeof(DeviceStatus), s) != cudaSuccess) return SHN_ERR_CUDA;
+  if (launch_decode_bf16(d_comp, comp_bytes, *p, st, d_out, out_elems, d_scales, log2_group, n_scales, sm_count(),
+                         s) != cudaSuccess)
+    return SHN_ERR_CUDA;
+  return SHN_OK;
+}
+
 int shn_get_device_status(const void* d_work, uint32_t* h_status, uint32_t* h_detail, void* stream) {
   if (!d_work || !h_status) return SHN_ERR_INVALID_ARG;
   DeviceStatus st;

@@ -26,6 +26,8 @@
 // Robustness. Corrupt input never causes an out-of-bounds access: descriptors and the chunk index
 // are validated against the stream and output sizes, the ring is filled only from the thread's own
 // chunk, and a decoded next-state row is always inside the table by construction.
+#include <cuda_bf16.h>
+
 #include "shn_internal.cuh"
 
 #ifndef DEC_WARPS
@@ -263,10 +265,93 @@ struct ChunkCtx {
   uint64_t cb;          // chunk start, bytes from the stream start
   uint32_t nw;          // chunk words
   uint32_t tbase;       // shared-window address of slot 0's entry for this thread (replica / plain table)
-  uint8_t* dst;         // where the chunk's first piece goes (FORMAT.md §6)
-  uint32_t dst_stride;  // bytes between consecutive pieces of the chunk (16 * chunks in its group)
+  uint64_t pos0;        // output position (symbols) of the chunk's first piece (FORMAT.md §6)
+  uint32_t pos_stride;  // symbols between consecutive pieces of the chunk (16 * chunks in its group)
   uint32_t pieces;
   uint32_t last_len;    // symbols in the last piece (1..16)
+};
+
+// Output sinks: where a chunk's decoded symbols go. Pieces are 16 consecutive output positions
+// (FORMAT.md §6); put_pair/put receive raw bytes in their low 8 bits (junk above).
+struct ByteSink {  // the INT8 tensor itself
+  uint8_t* out;
+  uint8_t* dst;
+  uint32_t stride;
+  bool aligned;
+  uint32_t ov[4];
+  __device__ __forceinline__ void start(const ChunkCtx& c) {
+    dst = out + c.pos0;
+    stride = c.pos_stride;
+    aligned = (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
+  }
+  __device__ __forceinline__ void begin_piece() {}
+  // pp and i are loop indices of fully unrolled loops, so they fold to constants
+  __device__ __forceinline__ void put_pair(int pp, uint32_t ba, uint32_t bb) {
+    const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
+    if ((pp & 1) == 0) ov[pp >> 1] = pair;
+    else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
+  }
+  __device__ __forceinline__ void put(int i, uint32_t b) {  // b's low byte into byte i % 4 of word i / 4
+    if ((i & 3) == 0) ov[i >> 2] = b;
+    else ov[i >> 2] = __byte_perm(ov[i >> 2], b, (i & 3) == 1 ? 0x3240u : (i & 3) == 2 ? 0x3410u : 0x4210u);
+  }
+  __device__ __forceinline__ void end_piece() {
+    if (aligned) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) dst[r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
+    }
+    dst += stride;
+  }
+  __device__ __forceinline__ void put_tail(uint32_t i, uint32_t b) { dst[i] = (uint8_t)b; }
+};
+
+// bf16 dequantisation fused into the decode: value = bf16_rn(float(int8) * scale[pos >> gshift]),
+// the product rounded once in fp32 as a separate multiply would. A piece lies in one scale group
+// (groups are >= 16 positions and pieces start at multiples of 16), so there is one scale load per
+// piece, issued one piece ahead.
+struct Bf16Sink {
+  uint16_t* out;
+  const float* scales;
+  uint32_t gshift;
+  uint64_t gmax;  // last valid scale index
+  uint64_t pos;
+  uint32_t stride;
+  float sc, sc_next;
+  uint32_t ov[4];
+  __device__ __forceinline__ void start(const ChunkCtx& c) {
+    pos = c.pos0;
+    stride = c.pos_stride;
+    sc_next = __ldg(scales + min(pos >> gshift, gmax));
+  }
+  __device__ __forceinline__ void begin_piece() {
+    sc = sc_next;
+    sc_next = __ldg(scales + min((pos + stride) >> gshift, gmax));  // the next piece's (clamped past the end)
+  }
+  static __device__ __forceinline__ float value(uint32_t b) {
+    // raw byte -> float(int8): 2^23 + (b ^ 0x80) as a float bit pattern, minus 2^23 + 128 (exact)
+    return __int_as_float(int((b & 0xFFu) ^ 0x4B000080u)) - 8388736.0f;
+  }
+  __device__ __forceinline__ uint32_t pack(uint32_t ba, uint32_t bb) const {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(value(ba) * sc, value(bb) * sc);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  // pp and i are loop indices of fully unrolled loops, so they fold to constants
+  __device__ __forceinline__ void put_pair(int pp, uint32_t ba, uint32_t bb) {
+    ov[pp & 3] = pack(ba, bb);
+    if ((pp & 3) == 3) *reinterpret_cast<uint4*>(out + pos + 8 * (pp >> 2)) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+  }
+  uint32_t held;
+  __device__ __forceinline__ void put(int i, uint32_t b) {
+    if ((i & 1) == 0) held = b;
+    else put_pair(i >> 1, held, b);
+  }
+  __device__ __forceinline__ void end_piece() { pos += stride; }
+  __device__ __forceinline__ void put_tail(uint32_t i, uint32_t b) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(value(b) * sc_next);  // the tail piece's scale
+    out[pos + i] = *reinterpret_cast<const uint16_t*>(&h);
+  }
 };
 
 // Ring fetcher: quads of 16 bytes (absolute, stream-relative), fetched downwards from the chunk end.
@@ -299,8 +384,8 @@ struct Fetcher {
 
 // One chunk. SH = log2 of the table row stride in bytes. PAIRS (fields <= 16 bits, L <= 256): two
 // symbols per window position; otherwise one (fields <= 20 bits).
-template <int S, int SH, bool PAIRS>
-__device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
+template <int S, int SH, bool PAIRS, class Sink>
+__device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink& sk) {
   const uint32_t mask = kRingBytes - 1;
   const uint32_t cb_mod = (uint32_t)(c.cb & mask);
   Fetcher fe;
@@ -336,14 +421,13 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
     P -= (int32_t)R;
     advance();
   }
-  const bool aligned = ((reinterpret_cast<uintptr_t>(c.dst) & 15u) == 0);
   const uint32_t full = c.pieces - (c.last_len < 16 ? 1u : 0u);
-  uint8_t* dst = c.dst;
-  for (uint32_t k = 0; k < full; ++k, dst += c.dst_stride) {
+  sk.start(c);
+  for (uint32_t k = 0; k < full; ++k) {
     fe.top_up<PAIRS ? 2 : 3>(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<1>();
-    uint32_t ov[4];
+    sk.begin_piece();
     if (!PAIRS) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -356,45 +440,35 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
         X[q] = E.x + r * (1u << SH);
         P = add_top_byte(E.y, P);
         advance();
-        const uint32_t b = add_shr16(E.y, o);
-        // b's low byte into byte i % 4 of the output word (the other bytes are kept)
-        if ((i & 3) == 0) ov[i >> 2] = b;
-        else ov[i >> 2] = __byte_perm(ov[i >> 2], b, (i & 3) == 1 ? 0x3240u : (i & 3) == 2 ? 0x3410u : 0x4210u);
+        sk.put(i, add_shr16(E.y, o));
       }
     } else {
 #pragma unroll
-    for (int pp = 0; pp < 8; ++pp) {
-      const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
-      const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);  // next 32 bits, top-aligned
-      const uint2 Ea = lds64(X[qa]);
-      const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);          // state bits: top nb of V
-      const uint32_t Va = __funnelshift_l(0u, V, Ea.y);          // V << nb
-      const uint32_t wa = shr8(Ea.y);                            // low 5 bits: w
-      const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
-      const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
-      const uint32_t ba = add_shr16(Ea.y, oa);                   // low byte: base' + offset
-      X[qa] = Ea.x + ra * (1u << SH);
-      P = add_top_byte(Ea.y, P);                                 // P -= nb + w
-      const uint2 Eb = lds64(X[qb]);
-      const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
-      const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
-      const uint32_t wb = shr8(Eb.y);
-      const uint32_t ob = __funnelshift_l(Vb, 0u, wb);
-      const uint32_t bb = add_shr16(Eb.y, ob);
-      X[qb] = Eb.x + rb * (1u << SH);
-      P = add_top_byte(Eb.y, P);
-      advance();
-      const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
-      if ((pp & 1) == 0) ov[pp >> 1] = pair;
-      else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
+      for (int pp = 0; pp < 8; ++pp) {
+        const int qa = (2 * pp) % S, qb = (2 * pp + 1) % S;
+        const uint32_t V = __funnelshift_r(W0, W1, (uint32_t)P);  // next 32 bits, top-aligned
+        const uint2 Ea = lds64(X[qa]);
+        const uint32_t ra = __funnelshift_l(V, 0u, Ea.y);          // state bits: top nb of V
+        const uint32_t Va = __funnelshift_l(0u, V, Ea.y);          // V << nb
+        const uint32_t wa = shr8(Ea.y);                            // low 5 bits: w
+        const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
+        const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
+        const uint32_t ba = add_shr16(Ea.y, oa);                   // low byte: base' + offset
+        X[qa] = Ea.x + ra * (1u << SH);
+        P = add_top_byte(Ea.y, P);                                 // P -= nb + w
+        const uint2 Eb = lds64(X[qb]);
+        const uint32_t rb = __funnelshift_l(V2, 0u, Eb.y);
+        const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
+        const uint32_t wb = shr8(Eb.y);
+        const uint32_t ob = __funnelshift_l(Vb, 0u, wb);
+        const uint32_t bb = add_shr16(Eb.y, ob);
+        X[qb] = Eb.x + rb * (1u << SH);
+        P = add_top_byte(Eb.y, P);
+        advance();
+        sk.put_pair(pp, ba, bb);
+      }
     }
-    }
-    if (aligned) {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-    } else {
-#pragma unroll
-      for (int r = 0; r < 16; ++r) dst[r] = (uint8_t)(ov[r >> 2] >> (8 * (r & 3)));
-    }
+    sk.end_piece();
   }
   if (full < c.pieces) {  // the group's short last piece
     fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
@@ -414,7 +488,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R) {
       x = E.x + r * (1u << SH);
       P = add_top_byte(E.y, P);
       advance();
-      dst[i] = (uint8_t)add_shr16(E.y, o);
+      sk.put_tail(i, add_shr16(E.y, o));
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;
@@ -439,9 +513,17 @@ __device__ __forceinline__ uint32_t segment_of(const uint8_t* descs, uint32_t n_
   return (uint32_t)a;
 }
 
-template <int S>
+// Output of a decode launch: INT8 bytes, or bf16 values dequantised by a scale per 2^gshift positions.
+struct DecOut {
+  uint8_t* out;
+  const float* scales;
+  uint32_t gshift;
+  uint64_t n_scales;
+};
+
+template <int S, bool BF16>
 __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(const uint8_t* __restrict__ comp, DeviceStatus* st,
-                                                             uint8_t* __restrict__ out) {
+                                                                             const DecOut o) {
   extern __shared__ __align__(128) unsigned char dsm[];
   if (*(volatile uint32_t*)&st->status != 0) return;
   const DecHeader h = read_header(comp);
@@ -459,6 +541,27 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
   }
   const uint64_t n_tiles = (h.total_chunks + kDecThreads - 1) / kDecThreads;
   int64_t cur_seg = -1;  // segment whose replicated table is in shared memory
+  const uint64_t gmax = h.total_symbols > 0 ? (h.total_symbols - 1) >> o.gshift : 0;
+  if (BF16 && h.total_symbols > 0 && gmax >= o.n_scales) {
+    if (blockIdx.x == 0 && tid == 0) report(st, SHN_ERR_CAPACITY, 0);
+    return;
+  }
+  // decode one chunk into the launch's output
+  auto run = [&](const ChunkCtx& cc, auto sh, auto pairs) -> bool {
+    constexpr int SH = decltype(sh)::value;
+    constexpr bool PAIRS = decltype(pairs)::value;
+    if (BF16) {
+      Bf16Sink sk;
+      sk.out = reinterpret_cast<uint16_t*>(o.out);
+      sk.scales = o.scales;
+      sk.gshift = o.gshift;
+      sk.gmax = gmax;
+      return decode_chunk<S, SH, PAIRS>(cc, h.R, sk);
+    }
+    ByteSink sk;
+    sk.out = o.out;
+    return decode_chunk<S, SH, PAIRS>(cc, h.R, sk);
+  };
 
   for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     const uint64_t g0 = tile * kDecThreads;
@@ -487,10 +590,14 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
         c.cb = h.payload_off + pay_start + 4ull * w0;
         c.nw = w1 - w0;
         const ChunkGeo geo = chunk_geo(n, h.C, ci);
-        c.dst = out + out_off + geo.base + 16u * geo.j;
-        c.dst_stride = 16u * geo.m;
+        c.pos0 = out_off + geo.base + 16u * geo.j;
+        c.pos_stride = 16u * geo.m;
         c.pieces = geo.pieces;
         c.last_len = geo.last_len;
+        if (BF16 && (out_off & 15) != 0) {  // pieces would straddle scale groups
+          report(st, SHN_ERR_UNSUPPORTED, (uint32_t)g);
+          valid = false;
+        }
       }
     }
     if (sa == sb) {
@@ -502,12 +609,14 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
       if (valid) {
         c.tbase = dsm_saddr + (lane & (dec_replicas(h.R) - 1)) * 8;
         bool ok;
+        using F = std::false_type;
+        using T = std::true_type;
         switch (h.R) {  // row stride: 16 copies x 8 bytes up to L = 256, then 8, 4, 2, 1 copies
-          case 9: ok = decode_chunk<S, 6, false>(c, h.R); break;
-          case 10: ok = decode_chunk<S, 5, false>(c, h.R); break;
-          case 11: ok = decode_chunk<S, 4, false>(c, h.R); break;
-          case 12: ok = decode_chunk<S, 3, false>(c, h.R); break;
-          default: ok = decode_chunk<S, 7, true>(c, h.R); break;
+          case 9: ok = run(c, std::integral_constant<int, 6>(), F()); break;
+          case 10: ok = run(c, std::integral_constant<int, 5>(), F()); break;
+          case 11: ok = run(c, std::integral_constant<int, 4>(), F()); break;
+          case 12: ok = run(c, std::integral_constant<int, 3>(), F()); break;
+          default: ok = run(c, std::integral_constant<int, 7>(), T()); break;
         }
         if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
       }
@@ -519,7 +628,8 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
         build_decode_tables(recs, h, lay, s0, nt, false, dsm, dsm_saddr);
         if (valid && seg >= s0 && seg < s0 + nt) {
           c.tbase = dsm_saddr + (seg - s0) * L * 8;
-          const bool ok = h.R <= 8 ? decode_chunk<S, 3, true>(c, h.R) : decode_chunk<S, 3, false>(c, h.R);
+          const bool ok = h.R <= 8 ? run(c, std::integral_constant<int, 3>(), std::true_type())
+                                   : run(c, std::integral_constant<int, 3>(), std::false_type());
           if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
         }
       }
@@ -527,33 +637,49 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
   }
 }
 
-template <int S>
-static cudaError_t launch_decode_t(const uint8_t* d_comp, DeviceStatus* st, uint8_t* d_out, const shn_params& p,
+template <int S, bool BF16>
+static cudaError_t launch_decode_t(const uint8_t* d_comp, DeviceStatus* st, const DecOut& o, const shn_params& p,
                                    int sm_count, cudaStream_t s) {
   const SmemLayout lay = smem_layout(p.log2L, p.K);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<S, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)lay.total);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<S>, kDecThreads, lay.total);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<S, BF16>, kDecThreads, lay.total);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  decode_kernel<S><<<sm_count * per_sm, kDecThreads, lay.total, s>>>(d_comp, st, d_out);
+  decode_kernel<S, BF16><<<sm_count * per_sm, kDecThreads, lay.total, s>>>(d_comp, st, o);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
-                          uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s) {
+template <bool BF16>
+static cudaError_t launch_decode_mode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p,
+                                      DeviceStatus* st, const DecOut& o, uint64_t out_capacity, int sm_count,
+                                      cudaStream_t s) {
   decode_check_kernel<<<1, 256, 0, s>>>(d_comp, comp_bytes, p, st, out_capacity);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (p.states_per_chunk) {
-    case 1: return launch_decode_t<1>(d_comp, st, d_out, p, sm_count, s);
-    case 2: return launch_decode_t<2>(d_comp, st, d_out, p, sm_count, s);
-    case 4: return launch_decode_t<4>(d_comp, st, d_out, p, sm_count, s);
-    case 8: return launch_decode_t<8>(d_comp, st, d_out, p, sm_count, s);
-    case 16: return launch_decode_t<16>(d_comp, st, d_out, p, sm_count, s);
+    case 1: return launch_decode_t<1, BF16>(d_comp, st, o, p, sm_count, s);
+    case 2: return launch_decode_t<2, BF16>(d_comp, st, o, p, sm_count, s);
+    case 4: return launch_decode_t<4, BF16>(d_comp, st, o, p, sm_count, s);
+    case 8: return launch_decode_t<8, BF16>(d_comp, st, o, p, sm_count, s);
+    case 16: return launch_decode_t<16, BF16>(d_comp, st, o, p, sm_count, s);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
+                          uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s) {
+  const DecOut o{d_out, nullptr, 0u, 0ull};
+  return launch_decode_mode<false>(d_comp, comp_bytes, p, st, o, out_capacity, sm_count, s);
+}
+
+cudaError_t launch_decode_bf16(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
+                               uint16_t* d_out, uint64_t out_elems, const float* d_scales, uint32_t log2_group,
+                               uint64_t n_scales, int sm_count, cudaStream_t s) {
+  const DecOut o{reinterpret_cast<uint8_t*>(d_out), d_scales, log2_group, n_scales};
+  return launch_decode_mode<true>(d_comp, comp_bytes, p, st, o, out_elems, sm_count, s);
 }
 
 }  // namespace shn

@@ -303,8 +303,11 @@ __global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t
   }
 }
 
-// Single-pass mode: one warp per chunk copies its words from the slot to the final place (32
-// consecutive words per step, four steps in flight per lane).
+// Single-pass mode: one warp per chunk moves its words from the slot (16-byte aligned) to the final
+// place (4-byte aligned) in 16-byte pieces: lane l loads source quad j = j0 + l, takes quad j - 1
+// from lane l - 1 (or from lane 31 of the previous step) and assembles destination quad j shifted by
+// the destination's misalignment a; only the chunk's first and last destination quads, which it
+// shares with its neighbours, are written word by word.
 __global__ void __launch_bounds__(256) encode_compact_kernel(const EncodeLayout lay, EncodeWork w,
                                                              uint8_t* __restrict__ out) {
   if (*(volatile uint32_t*)&w.status->status != 0) return;
@@ -312,19 +315,45 @@ __global__ void __launch_bounds__(256) encode_compact_kernel(const EncodeLayout 
   const uint32_t lane = threadIdx.x & 31;
   const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
   for (uint64_t g = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < lay.total_chunks; g += warps) {
-    const uint32_t* __restrict__ src = w.slots + g * w.slot_words;
-    uint32_t* __restrict__ dst = payload + w.word_offset[g];
-    const uint32_t n = w.chunk_words[g];
-    uint32_t i = lane;
-    for (; i + 96 < n; i += 128) {
-      const uint32_t v0 = __ldcs(src + i), v1 = __ldcs(src + i + 32), v2 = __ldcs(src + i + 64),
-                     v3 = __ldcs(src + i + 96);
-      dst[i] = v0;
-      dst[i + 32] = v1;
-      dst[i + 64] = v2;
-      dst[i + 96] = v3;
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(w.slots + g * w.slot_words);
+    const uint64_t D = w.word_offset[g];
+    const uint32_t n = w.chunk_words[g];  // >= 1 (the sentinel)
+    const uint32_t a = (uint32_t)D & 3u;
+    const uint64_t q0 = D >> 2;
+    const uint32_t nq = (uint32_t)(((D + n - 1) >> 2) - q0 + 1);
+    uint4 carry = make_uint4(0u, 0u, 0u, 0u);
+    for (uint32_t j0 = 0; j0 < nq; j0 += 32) {
+      const uint32_t j = j0 + lane;
+      const uint4 cur = (4 * j < n) ? __ldcs(src + j) : make_uint4(0u, 0u, 0u, 0u);
+      uint4 prv;
+      prv.x = __shfl_up_sync(0xffffffffu, cur.x, 1);
+      prv.y = __shfl_up_sync(0xffffffffu, cur.y, 1);
+      prv.z = __shfl_up_sync(0xffffffffu, cur.z, 1);
+      prv.w = __shfl_up_sync(0xffffffffu, cur.w, 1);
+      if (lane == 0) prv = carry;
+      carry.x = __shfl_sync(0xffffffffu, cur.x, 31);
+      carry.y = __shfl_sync(0xffffffffu, cur.y, 31);
+      carry.z = __shfl_sync(0xffffffffu, cur.z, 31);
+      carry.w = __shfl_sync(0xffffffffu, cur.w, 31);
+      if (j < nq) {
+        uint4 o;
+        switch (a) {  // warp-uniform
+          case 0: o = cur; break;
+          case 1: o = make_uint4(prv.w, cur.x, cur.y, cur.z); break;
+          case 2: o = make_uint4(prv.z, prv.w, cur.x, cur.y); break;
+          default: o = make_uint4(prv.y, prv.z, prv.w, cur.x); break;
+        }
+        const uint64_t d0 = 4 * (q0 + j);  // first destination word of this quad
+        if (d0 >= D && d0 + 4 <= D + n) {
+          *reinterpret_cast<uint4*>(payload + d0) = o;
+        } else {
+          const uint32_t ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (d0 + t >= D && d0 + t < D + n) payload[d0 + t] = ov[t];
+        }
+      }
     }
-    for (; i < n; i += 32) dst[i] = __ldcs(src + i);
   }
 }
 

@@ -209,5 +209,8 @@ cudaError_t launch_encode_compact(const EncodeLayout& lay, const EncodeWork& w, 
 
 cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
                           uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s);
+cudaError_t launch_decode_bf16(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
+                               uint16_t* d_out, uint64_t out_elems, const float* d_scales, uint32_t log2_group,
+                               uint64_t n_scales, int sm_count, cudaStream_t s);
 
 }  // namespace shn

@@ -58,12 +58,13 @@ def weight_like_int8(rows: int = 4096, cols: int = 1024, seed: int = 1, device="
     return torch.round(w / scale).clamp_(-127, 127).to(torch.int8).reshape(-1)
 
 
-def kv_cache_segment_int8(layer: int, kv: int, seed: int = 2, device="cpu", shape=KV_SHAPE) -> torch.Tensor:
-    """One (layer, K/V) slice of the INT8 KV cache [layers, 2, batch, kv_heads, seq, head_dim].
+def kv_cache_segment_int8_and_scales(layer: int, kv: int, seed: int = 2, device="cpu", shape=KV_SHAPE):
+    """One (layer, K/V) slice of the INT8 KV cache [layers, 2, batch, kv_heads, seq, head_dim] and
+    its dequantisation scales (float32, one per head_dim group, in group order).
 
     bf16 N(0,1) values times a per-channel scale ~ LogNormal(0, 0.5) (a channel is a
     (layer, K/V, kv_head, head_dim) position, shared over batch and seq), then absmax INT8
-    quantisation per group of head_dim (=128) values.
+    quantisation per group of head_dim (=128) values: q = round(x / s), s = absmax / 127.
     """
     _, _, B, Hk, T, D = shape
     g = _gen(seed * 1_000_003 + layer * 2 + kv, device)
@@ -71,7 +72,13 @@ def kv_cache_segment_int8(layer: int, kv: int, seed: int = 2, device="cpu", shap
     x = torch.randn(B, Hk, T, D, generator=g, device=device)
     x = (x * scale[None, :, None, :]).to(torch.bfloat16).float()
     s = x.abs().amax(dim=-1, keepdim=True).clamp_min(1e-30) / 127.0
-    return torch.round(x / s).clamp_(-127, 127).to(torch.int8).reshape(-1)
+    q = torch.round(x / s).clamp_(-127, 127).to(torch.int8).reshape(-1)
+    return q, s.reshape(-1).float()
+
+
+def kv_cache_segment_int8(layer: int, kv: int, seed: int = 2, device="cpu", shape=KV_SHAPE) -> torch.Tensor:
+    """The INT8 values of kv_cache_segment_int8_and_scales."""
+    return kv_cache_segment_int8_and_scales(layer, kv, seed, device, shape)[0]
 
 
 def kv_cache_int8(seed: int = 2, device="cpu", shape=KV_SHAPE) -> torch.Tensor:
@@ -85,6 +92,13 @@ def kv_cache_int8(seed: int = 2, device="cpu", shape=KV_SHAPE) -> torch.Tensor:
             i = layer * KV + kv
             out[i * seg:(i + 1) * seg] = kv_cache_segment_int8(layer, kv, seed, device, shape)
     return out
+
+
+def kv_cache_scales(seed: int = 2, device="cpu", shape=KV_SHAPE) -> torch.Tensor:
+    """Dequantisation scales of kv_cache_int8 (one float32 per head_dim group, in tensor order)."""
+    L, KV = shape[0], shape[1]
+    return torch.cat([kv_cache_segment_int8_and_scales(layer, kv, seed, device, shape)[1]
+                      for layer in range(L) for kv in range(KV)])
 
 
 def kv_cache_segments(shape=KV_SHAPE):

@@ -29,7 +29,7 @@ TABLE_PUBLIC_BYTES = 800
 EXPORTED = [
     "shn_version", "shn_status_string", "shn_check_params", "shn_table_bytes", "shn_encode_bound",
     "shn_encode_workspace_bytes", "shn_encode_workspace_bytes_min", "shn_decode_workspace_bytes", "shn_histogram", "shn_build_tables",
-    "shn_encode", "shn_decode", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
+    "shn_encode", "shn_decode", "shn_decode_bf16", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
 ]
 
 
@@ -84,6 +84,7 @@ def lib():
             "shn_build_tables": (i32, [vp, u32, P, vp, vp]),
             "shn_encode": (i32, [vp, vp, u32, vp, P, vp, sz, vp, sz, vp, vp]),
             "shn_decode": (i32, [vp, sz, P, vp, sz, vp, sz, vp]),
+            "shn_decode_bf16": (i32, [vp, sz, P, vp, sz, u32, vp, sz, vp, sz, vp]),
             "shn_get_device_status": (i32, [vp, ctypes.POINTER(u32), ctypes.POINTER(u32), vp]),
             "shn_encode_static_max_chunks": (u64, []),
             "shn_encode_static": (i32, [vp, vp, u32, vp, P, vp, sz, vp, vp, vp]),
@@ -211,6 +212,17 @@ def shn_decode(comp: torch.Tensor, comp_bytes: int, p: CodecParams, work: torch.
     _check(lib().shn_decode(_dev(comp, "comp"), int(comp_bytes), ctypes.byref(p.c()), _dev(work, "work"),
                             work.numel(), _dev(out, "out") if out.numel() else None, out.numel(),
                             _stream(stream)), "shn_decode")
+
+
+def shn_decode_bf16(comp: torch.Tensor, comp_bytes: int, p: CodecParams, scales: torch.Tensor, log2_group: int,
+                    work: torch.Tensor, out: torch.Tensor, stream=None):
+    """Decode fused with dequantisation: out (bfloat16) = int8 value x scales[i >> log2_group]."""
+    if scales.dtype != torch.float32 or out.dtype != torch.bfloat16:
+        raise ValueError("scales must be float32 and out bfloat16")
+    _check(lib().shn_decode_bf16(_dev(comp, "comp"), int(comp_bytes), ctypes.byref(p.c()), _dev(scales, "scales"),
+                                 scales.numel(), int(log2_group), _dev(work, "work"), work.numel(),
+                                 _dev(out, "out") if out.numel() else None, out.numel(), _stream(stream)),
+           "shn_decode_bf16")
 
 
 def shn_get_device_status(work: torch.Tensor, stream=None):

@@ -173,6 +173,24 @@ int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, vo
                uint8_t* d_out, size_t out_capacity, void* stream);
 
 /*
+ * Decode fused with the consumer's dequantisation: instead of the INT8 tensor, write
+ *   d_out[i] = bf16_rn( float(int8 value i) * d_scales[i >> log2_group] )
+ * (the product rounded once in fp32, then to bfloat16 round-to-nearest-even), e.g. a KV cache
+ * quantised with one absmax scale per head_dim group. Saves the INT8 write-back and the separate
+ * dequantisation pass (Shannonic §6.2: compression for KV/activation transfer; the paper decodes
+ * to INT8 and has no fused form).
+ *  d_scales    device float[n_scales], 4-byte aligned; n_scales >= ceil(total_symbols / 2^log2_group).
+ *  log2_group  4 <= log2_group <= 31 (groups of >= 16 positions).
+ *  d_out       device, out_elems bfloat16 values (as uint16), 16-byte aligned.
+ * Every segment must start at an output position that is a multiple of 16 (device status
+ * SHN_ERR_UNSUPPORTED otherwise). Other arguments, errors and status as in shn_decode; too few
+ * scales gives device status SHN_ERR_CAPACITY.
+ */
+int shn_decode_bf16(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, const float* d_scales,
+                    size_t n_scales, uint32_t log2_group, void* d_work, size_t work_bytes, uint16_t* d_out,
+                    size_t out_elems, void* stream);
+
+/*
  * shn_encode without a workspace, for callers that cannot allocate device memory. (This entry
  * point is an addition of this library; the paper has no counterpart.)
  *
