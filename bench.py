@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused decode+dequantise measurement (kv)")
+    ap.add_argument("--no-offload", action="store_true", help="skip the host offload/reload measurement (kv)")
     ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
     ap.add_argument("--entropy", type=float, default=5.3, choices=[2.0, 4.0, 5.3, 7.9], help="sweep workload")
     ap.add_argument("--K", type=int, default=None, help="override the workload's range count")
@@ -537,6 +538,63 @@ def main():
                  "unfused_ms": ms_u, "unfused": "shn_decode then (int8.float() * scale).to(bfloat16) in PyTorch",
                  "speedup_vs_unfused": ms_u / ms_f, "matches_unfused": bool(fused_ok)}
 
+    # Compressed offload to host memory and pipelined reload (8 streams of 8 segments each), against
+    # plain pinned copies of the INT8 tensor over the same link.
+    offl = None
+    if args.workload == "kv" and not args.segments and not args.no_offload:
+        ends = list(range(8, len(segs) + 1, 8))
+        batches = [segs[a:b] for a, b in zip([0] + ends[:-1], ends)]
+        owork = shn.empty_aligned(shn.offload_workspace_bytes(p, segs, ends), dev)
+        h_all = torch.empty(comp_cap + 16 * len(batches), dtype=torch.uint8, pin_memory=True)
+        h_raw = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+        wrk = shn.empty_aligned(256, dev)
+        back = torch.empty(n, dtype=torch.uint8, device=dev)
+        copy_stream = torch.cuda.Stream(dev)
+        placed = {}
+
+        def do_offload():  # blocks until the last batch is encoded; the copies finish on copy_stream
+            placed["offs"], placed["sizes"] = shn.shn_offload(x, segs, ends, p, owork, h_all, stream, copy_stream)
+            stream.wait_stream(copy_stream)
+
+        do_offload()
+        torch.cuda.synchronize()
+        sizes = placed["sizes"]
+        hosts = [h_all[o:o + b] for o, b in zip(placed["offs"], sizes)]
+        offsets = np.cumsum([0] + [sum(ln for _, ln in b) for b in batches])[:-1].tolist()
+        staging = shn.empty_aligned(2 * max(-(-v // 16) * 16 for v in sizes), dev, 16)
+
+        def do_reload():
+            shn.shn_decode_from_host(hosts, sizes, p, staging, wrk, back, offsets, stream, copy_stream)
+
+        def ev_time(fn, reps=3):
+            fn()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            return sorted(ts)[len(ts) // 2]
+
+        ms_off = ev_time(do_offload)
+        ms_rel = ev_time(do_reload)
+        reload_ok = shn.shn_get_device_status(wrk)[0] == 0 and torch.equal(back, x.view(torch.uint8))
+        ms_d2h = ev_time(lambda: h_raw.copy_(x.view(torch.uint8), non_blocking=True))
+        ms_h2d = ev_time(lambda: back.copy_(h_raw, non_blocking=True))
+        comp = sum(sizes)
+        offl = {"what": "shn_offload: 8 streams of 8 segments, each copied to pinned host memory by the copy engine "
+                        "while the next encodes; shn_decode_from_host copying them back while the previous decodes",
+                "compressed_bytes": comp, "int8_bytes": n,
+                "offload_ms": ms_off, "offload_gbs_int8": n / (ms_off * 1e-3) / 1e9,
+                "reload_ms": ms_rel, "reload_gbs_int8": n / (ms_rel * 1e-3) / 1e9,
+                "raw_d2h_ms": ms_d2h, "raw_h2d_ms": ms_h2d,
+                "offload_vs_raw": ms_d2h / ms_off, "reload_vs_raw": ms_h2d / ms_rel,
+                "reload_correct": bool(reload_ok)}
+        del hosts, h_all, h_raw, staging, back, owork
+
     if rank == 0:
         peak, peak_kind = measured_peaks()
         if fused is not None:
@@ -589,6 +647,7 @@ def main():
             "correct": bool(ok),
             "clocks": clk.summary(),
             "decode_bf16_fused": fused,
+            "offload": offl,
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
         }

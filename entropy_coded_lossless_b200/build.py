@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libshn.so")
-SOURCES = ["capi.cu", "histogram.cu", "build_tables.cu", "encode.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["capi.cu", "histogram.cu", "build_tables.cu", "encode.cu", "decode.cu", "noalloc.cu", "offload.cu"]
 HEADERS = [os.path.join(CSRC, "shn_internal.cuh"), os.path.join(ROOT, "include", "shn.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

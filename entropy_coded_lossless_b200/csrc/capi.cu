@@ -35,12 +35,7 @@ bool segs_ok(const shn_segment* segs, uint32_t n, uint64_t* total_chunks, uint64
   return true;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
+int sm_count() { return sm_count_for_launch(); }
 
 // Encode workspace: status word, per-chunk word counts, their exclusive prefix, scan block sums
 // (`total`, enough for the two-pass encoder); then, for the single-pass encoder, one worst-case

@@ -77,6 +77,14 @@ __device__ __forceinline__ const uint16_t* table_enc(const shn_table* t) {
   return reinterpret_cast<const uint16_t*>(t->opaque + kOpaqueEncOffset);
 }
 
+// SMs of the current device (grid sizing of the persistent kernels).
+inline int sm_count_for_launch() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
 // Encoder block size: one thread per chunk, so also the chunks each encoder block codes. The host
 // batching (block_start) and the encoder kernels both use it.
 #ifndef ENC_THREADS

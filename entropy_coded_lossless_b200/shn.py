@@ -29,7 +29,8 @@ TABLE_PUBLIC_BYTES = 800
 EXPORTED = [
     "shn_version", "shn_status_string", "shn_check_params", "shn_table_bytes", "shn_encode_bound",
     "shn_encode_workspace_bytes", "shn_encode_workspace_bytes_min", "shn_decode_workspace_bytes", "shn_histogram", "shn_build_tables",
-    "shn_encode", "shn_decode", "shn_decode_bf16", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
+    "shn_encode", "shn_decode", "shn_decode_bf16", "shn_decode_from_host", "shn_offload_workspace_bytes",
+    "shn_offload", "shn_get_device_status", "shn_encode_static_max_chunks", "shn_encode_static",
 ]
 
 
@@ -85,6 +86,11 @@ def lib():
             "shn_encode": (i32, [vp, vp, u32, vp, P, vp, sz, vp, sz, vp, vp]),
             "shn_decode": (i32, [vp, sz, P, vp, sz, vp, sz, vp]),
             "shn_decode_bf16": (i32, [vp, sz, P, vp, sz, u32, vp, sz, vp, sz, vp]),
+            "shn_offload_workspace_bytes": (sz, [P, vp, ctypes.POINTER(u32), u32]),
+            "shn_offload": (i32, [vp, vp, ctypes.POINTER(u32), u32, P, vp, sz, vp, sz, ctypes.POINTER(sz),
+                                  ctypes.POINTER(sz), vp, vp]),
+            "shn_decode_from_host": (i32, [ctypes.POINTER(vp), ctypes.POINTER(sz), u32, P, vp, sz, vp, sz, vp,
+                                           ctypes.POINTER(sz), sz, vp, vp]),
             "shn_get_device_status": (i32, [vp, ctypes.POINTER(u32), ctypes.POINTER(u32), vp]),
             "shn_encode_static_max_chunks": (u64, []),
             "shn_encode_static": (i32, [vp, vp, u32, vp, P, vp, sz, vp, vp, vp]),
@@ -116,9 +122,11 @@ def _segments(segments):
     return arr
 
 
-def _dev(t: torch.Tensor, name: str) -> int:
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+def _dev(t: torch.Tensor, name: str, host_ok: bool = False) -> int:
+    """Device address of t; with host_ok, pinned host memory (mapped into the device address space)
+    is accepted too."""
+    if not isinstance(t, torch.Tensor) or not (t.is_cuda or (host_ok and t.is_pinned())):
+        raise ValueError(f"{name} must be a CUDA tensor" + (" or pinned host memory" if host_ok else ""))
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
@@ -189,7 +197,7 @@ def shn_encode(x: torch.Tensor, segments, tables: torch.Tensor, p: CodecParams, 
     xb = _bytes_view(x)
     _check(lib().shn_encode(_dev(xb, "x") if xb.numel() else (xb.data_ptr() or None), _segments(segments),
                             len(segments), _dev(tables, "tables") if tables.numel() else None, ctypes.byref(p.c()),
-                            _dev(work, "work"), work.numel(), _dev(out, "out"), out.numel(),
+                            _dev(work, "work"), work.numel(), _dev(out, "out", host_ok=True), out.numel(),
                             _dev(out_bytes, "out_bytes"), _stream(stream)), "shn_encode")
 
 
@@ -223,6 +231,44 @@ def shn_decode_bf16(comp: torch.Tensor, comp_bytes: int, p: CodecParams, scales:
                                  scales.numel(), int(log2_group), _dev(work, "work"), work.numel(),
                                  _dev(out, "out") if out.numel() else None, out.numel(), _stream(stream)),
            "shn_decode_bf16")
+
+
+def offload_workspace_bytes(p: CodecParams, segments, batch_ends) -> int:
+    ends = (ctypes.c_uint32 * len(batch_ends))(*[int(e) for e in batch_ends])
+    return int(lib().shn_offload_workspace_bytes(ctypes.byref(p.c()), _segments(segments), ends, len(batch_ends)))
+
+
+def shn_offload(x: torch.Tensor, segments, batch_ends, p: CodecParams, work: torch.Tensor, h_out: torch.Tensor,
+                stream=None, copy_stream=None):
+    """Offload x as one SHN1 stream per batch of segments into pinned host memory h_out; returns
+    (offsets, sizes) of the streams in h_out. Blocks until the last batch is encoded."""
+    if h_out.device.type != "cpu" or h_out.dtype != torch.uint8:
+        raise ValueError("h_out must be a uint8 CPU tensor")
+    nb = len(batch_ends)
+    ends = (ctypes.c_uint32 * nb)(*[int(e) for e in batch_ends])
+    offs, sizes = (ctypes.c_size_t * nb)(), (ctypes.c_size_t * nb)()
+    xb = _bytes_view(x)
+    _check(lib().shn_offload(_dev(xb, "x"), _segments(segments), ends, nb, ctypes.byref(p.c()), _dev(work, "work"),
+                             work.numel(), h_out.data_ptr(), h_out.numel(), offs, sizes, _stream(stream),
+                             _stream(copy_stream if copy_stream is not None else stream)), "shn_offload")
+    return list(offs), list(sizes)
+
+
+def shn_decode_from_host(h_streams, stream_bytes, p: CodecParams, staging: torch.Tensor, work: torch.Tensor,
+                         out: torch.Tensor, out_offsets, stream=None, copy_stream=None):
+    """Pipelined reload: copy each host stream (pinned uint8 tensors) to `staging` on copy_stream
+    while the previous one decodes into out[out_offsets[i]:] on stream."""
+    n = len(h_streams)
+    for t in h_streams:
+        if t.device.type != "cpu" or t.dtype != torch.uint8:
+            raise ValueError("host streams must be uint8 CPU tensors")
+    ptrs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in h_streams])
+    sizes = (ctypes.c_size_t * n)(*[int(b) for b in stream_bytes])
+    offs = (ctypes.c_size_t * n)(*[int(o) for o in out_offsets])
+    _check(lib().shn_decode_from_host(ptrs, sizes, n, ctypes.byref(p.c()), _dev(staging, "staging"), staging.numel(),
+                                      _dev(work, "work"), work.numel(), _dev(out, "out"), offs, out.numel(),
+                                      _stream(stream), _stream(copy_stream if copy_stream is not None else stream)),
+           "shn_decode_from_host")
 
 
 def shn_get_device_status(work: torch.Tensor, stream=None):

@@ -145,7 +145,9 @@ int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params
  *  d_work        device workspace of >= shn_encode_workspace_bytes_min(p, h_segs, n_segs) bytes,
  *                256-byte aligned; >= shn_encode_workspace_bytes(...) selects the single-pass
  *                mode (same output). Its first 8 bytes receive the device status.
- *  d_out         device, out_capacity bytes, 16-byte aligned; receives the stream.
+ *  d_out         device, out_capacity bytes, 16-byte aligned; receives the stream. May be pinned
+ *                host memory mapped into the device address space (offload): with the
+ *                single-pass workspace the compressed bytes then cross the link exactly once.
  *  d_out_bytes   device uint64: the stream size in bytes (written even when it exceeds the
  *                capacity, in which case the device status is SHN_ERR_CAPACITY and d_out holds
  *                no complete stream).
@@ -189,6 +191,49 @@ int shn_decode(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, vo
 int shn_decode_bf16(const uint8_t* d_comp, size_t comp_bytes, const shn_params* p, const float* d_scales,
                     size_t n_scales, uint32_t log2_group, void* d_work, size_t work_bytes, uint16_t* d_out,
                     size_t out_elems, void* stream);
+
+/*
+ * Pipelined offload of a device tensor into host memory as n_batches SHN1 streams, one per batch of
+ * segments (batch b = h_segs[batch_ends[b-1] .. batch_ends[b]), batch_ends[-1] = 0): for each batch
+ * histogram, tables and encode run on `stream` into a device staging buffer; as soon as batch b is
+ * encoded the host reads its size and the copy engine moves exactly that many bytes to
+ * h_out + h_stream_offsets[b] on `copy_stream`, while batch b+1 encodes. Streams are placed back to
+ * back at 16-byte boundaries. Shannonic §6.2 (compression for transfers); no counterpart in the
+ * paper's code. The call blocks the host until the last batch is encoded; the copies complete in
+ * `copy_stream` order.
+ *  d_work   device workspace of >= shn_offload_workspace_bytes(...) bytes, 256-byte aligned.
+ *  h_out    host, h_capacity bytes (pinned for asynchronous copies).
+ *  h_stream_offsets, h_stream_bytes  host arrays of n_batches, filled by the call.
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_WORKSPACE, SHN_ERR_CAPACITY (h_out too small), SHN_ERR_CUDA,
+ *         or an encoder's device status (then the batches after it are not offloaded).
+ */
+size_t shn_offload_workspace_bytes(const shn_params* p, const shn_segment* h_segs, const uint32_t* batch_ends,
+                                   uint32_t n_batches);
+int shn_offload(const uint8_t* d_in, const shn_segment* h_segs, const uint32_t* batch_ends, uint32_t n_batches,
+                const shn_params* p, void* d_work, size_t work_bytes, uint8_t* h_out, size_t h_capacity,
+                size_t* h_stream_offsets, size_t* h_stream_bytes, void* stream, void* copy_stream);
+
+/*
+ * Pipelined reload of a tensor offloaded as n_streams SHN1 streams in host memory (e.g. written by
+ * shn_encode into pinned host buffers, one stream per batch of segments): stream i is copied to a
+ * device staging buffer on `copy_stream` (the copy engine) while stream i-1 decodes on `stream`,
+ * into d_out + out_offsets[i]. Shannonic §6.2: a transfer carries r/8 instead of 1 byte per value,
+ * which pays off when decoding keeps up with the link. No counterpart in the paper's code.
+ *  h_streams[i]   host, stream_bytes[i] bytes (pinned for an asynchronous copy); read on the host
+ *                 for its header (magic, symbol count) before anything is enqueued.
+ *  d_staging      device, staging_bytes >= 2 * round_up(max stream_bytes[i], 16), 16-byte aligned.
+ *  d_work         device workspace of >= 256 bytes (shared status word of all the decodes).
+ *  d_out          device, out_capacity bytes; stream i's symbols go to [out_offsets[i], +its count).
+ *  stream, copy_stream  the decode and copy streams (may be the same: then nothing overlaps).
+ * Returns when everything is enqueued; the work completes in `stream` order.
+ * Errors: SHN_ERR_INVALID_ARG, SHN_ERR_CORRUPT (a header that is not SHN1), SHN_ERR_CAPACITY (an
+ *         output range outside d_out), SHN_ERR_WORKSPACE (staging too small), SHN_ERR_CUDA;
+ *         device: as shn_decode (the first error of any stream).
+ */
+int shn_decode_from_host(const uint8_t* const* h_streams, const size_t* stream_bytes, uint32_t n_streams,
+                         const shn_params* p, uint8_t* d_staging, size_t staging_bytes, void* d_work,
+                         size_t work_bytes, uint8_t* d_out, const size_t* out_offsets, size_t out_capacity,
+                         void* stream, void* copy_stream);
 
 /*
  * shn_encode without a workspace, for callers that cannot allocate device memory. (This entry
