@@ -58,6 +58,20 @@ def weight_like_int8(rows: int = 4096, cols: int = 1024, seed: int = 1, device="
     return torch.round(w / scale).clamp_(-127, 127).to(torch.int8).reshape(-1)
 
 
+def int4_weight_like(rows: int = 4096, cols: int = 4096, group: int = 64, seed: int = 6, device="cpu") -> torch.Tensor:
+    """INT4 group-wise quantised weight-like tensor, one value per byte (int8 in [-8, 7]).
+
+    N(0,1) weights with 1% outliers x8 (as weight_like_int8), absmax-quantised to the symmetric
+    4-bit grid per group of `group` consecutive values of a row: q = clamp(round(w / s), -8, 7),
+    s = absmax / 7. The 4-bit alphabet enters the codec as 16 symbols of the byte alphabet."""
+    g = _gen(seed, device)
+    w = torch.randn(rows, cols, generator=g, device=device)
+    mask = torch.rand(rows, cols, generator=g, device=device) < 0.01
+    w = torch.where(mask, w * 8.0, w).reshape(rows, cols // group, group)
+    s = w.abs().amax(dim=-1, keepdim=True).clamp_min(1e-30) / 7.0
+    return torch.round(w / s).clamp_(-8, 7).to(torch.int8).reshape(-1)
+
+
 def kv_cache_segment_int8_and_scales(layer: int, kv: int, seed: int = 2, device="cpu", shape=KV_SHAPE):
     """One (layer, K/V) slice of the INT8 KV cache [layers, 2, batch, kv_heads, seq, head_dim] and
     its dequantisation scales (float32, one per head_dim group, in group order).

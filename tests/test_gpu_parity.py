@@ -93,6 +93,14 @@ def test_config2_weight_like(orc):
     check_parity(orc, x, [(0, x.size)], shn.CodecParams(16, 7, 4096, 4))
 
 
+def test_int4_weights(orc):
+    """INT4 group-quantised weights, one value per byte: a 16-symbol alphabet inside the byte one."""
+    x = inputs.int4_weight_like(512, 2048, seed=6).numpy()
+    g, _ = check_parity(orc, x, [(0, x.size)], shn.CodecParams(16, 7, 4096, 4))
+    st = spec.parse_stream(g["stream"])
+    assert st["segments"][0]["payload_words"] * 32 < 4 * x.size  # below 4 bits per weight
+
+
 def test_config2_plain_tans_l1024(orc):
     """The comparator of the weight-tensor config: plain tANS (K = 256 identity ranges) at L = 1024,
     bit-exact on the GPU, and (as on the pages) longer than Shannonic K = 16, L = 128."""
