@@ -74,14 +74,14 @@ __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L
           }
         }
       }
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long og = __shfl_xor_sync(0xffffffffu, bg, o);
-        const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        if (ok != 0x7fffffff && (bk == 0x7fffffff || og > bg || (og == bg && ok < bk))) {
-          bg = og;
-          bk = ok;
-        }
-      }
+      // warp argmax of (gain, then smallest k) with three reductions: the high word of the gain,
+      // the low word among lanes at that high word, the smallest k among lanes at the maximum.
+      // Every valid gain is > 0 (N_k > 0 and LG strictly increasing), lanes without one hold 0.
+      const uint32_t ghi = (uint32_t)(bg >> 32), glo = (uint32_t)bg;
+      const uint32_t m1 = __reduce_max_sync(0xffffffffu, ghi);
+      const uint32_t m2 = __reduce_max_sync(0xffffffffu, ghi == m1 ? glo : 0u);
+      bk = (int)__reduce_min_sync(0xffffffffu, (ghi == m1 && glo == m2 && bk != 0x7fffffff) ? (uint32_t)bk
+                                                                                                 : 0xffffffffu);
 #pragma unroll
       for (int r = 0; r < kPer; ++r)
         if (tid + 32 * r == bk) f[r] += 1;
@@ -154,13 +154,13 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
       atomicAdd(reinterpret_cast<unsigned long long*>(&S.cost), 0ull - (unsigned long long)n * lg_fixed(n));
     }
   } else {
-    for (int q = tid; q < kPairs; q += kBuildThreads) {
-      int i = (int)((1.0f + sqrtf(8.0f * (float)q + 1.0f)) * 0.5f);
-      while (i * (i - 1) / 2 > q) --i;
-      while ((i + 1) * i / 2 <= q) ++i;
-      const int j = q - i * (i - 1) / 2;
-      // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30
-      lgc[q] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) - (int32_t)lg_fixed(S.pre[i] - S.pre[j]));
+    // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30; warp w
+    // fills the rows i = w+1, w+17, ... (about the same number of pairs per warp)
+    for (int i = 1 + (tid >> 5); i <= 256; i += kBuildThreads / 32) {
+      const uint32_t pi = S.pre[i];
+      uint32_t* row = lgc + i * (i - 1) / 2;
+      for (int j = tid & 31; j < i; j += 32)
+        row[j] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) - (int32_t)lg_fixed(pi - S.pre[j]));
     }
     for (int i = tid; i <= 256; i += kBuildThreads) S.drow[0][i] = (i == 0) ? 0 : LLONG_MAX;
     __syncthreads();
@@ -179,18 +179,19 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
       int bj_a = 0x7fffffff, bj_b = 0x7fffffff;
       const uint32_t pa = S.pre[ia], pb = S.pre[ib];
       const int base_a = ia * (ia - 1) / 2, base_b = ib * (ib - 1) / 2;
-      for (int t = r4; t < na + nb; t += 4) {
-        const bool in_a = t < na;
-        const int j = (k - 1) + (in_a ? t : t - na);
-        const uint32_t c = (in_a ? pa : pb) - S.pre[j];
-        const int32_t d = (int32_t)lgc[(in_a ? base_a : base_b) + j];
-        const long long v = prev[j] + (long long)c * (long long)d;  // Cost(j, i-1) = c * (w << 24) - c * LG(c)
-        if (in_a) {
-          if (v < best_a) {
-            best_a = v;
-            bj_a = j;
-          }
-        } else if (v < best_b) {
+      // Cost(j, i-1) = c * (w << 24) - c * LG(c) = c * lgc[pair]; each thread takes every 4th start
+      for (int t = r4; t < na; t += 4) {
+        const int j = (k - 1) + t;
+        const long long v = prev[j] + (long long)(pa - S.pre[j]) * (long long)(int32_t)lgc[base_a + j];
+        if (v < best_a) {
+          best_a = v;
+          bj_a = j;
+        }
+      }
+      for (int t = r4; t < nb; t += 4) {
+        const int j = (k - 1) + t;
+        const long long v = prev[j] + (long long)(pb - S.pre[j]) * (long long)(int32_t)lgc[base_b + j];
+        if (v < best_b) {
           best_b = v;
           bj_b = j;
         }
