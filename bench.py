@@ -134,7 +134,7 @@ MEASURED_TRAFFIC = {
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0001,
         "source": "build_tables.cu",
-        "sha256_prefix": "815cc03fefc83892"
+        "sha256_prefix": "4da24da9e6f46b0d"
     },
     "encode_compact_kernel": {
         "bytes_per_symbol": 1.7817,
