@@ -112,47 +112,57 @@ def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
 
 
 # DRAM bytes (read + write) per symbol of each kernel, from the ncu captures summarised in
-# profiles/<kernel>_kv_cache_1GiB.md (KV cache, K=16, L=128, C=4096, S=4), with the sha256 prefix of
-# the kernel's source file at capture time: if the source has changed since, the figure is stale and
-# the bench reports traffic as null.
+# profiles/<kernel>_kv_cache_1GiB.md (KV cache, K=16, L=128, C=4096, S=4), with the digest of the
+# kernel's source file (comments removed) at capture time: if the code has changed since, the figure
+# is stale and the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     "decode_kernel": {
         "bytes_per_symbol": 1.8894,
         "source": "decode.cu",
-        "sha256_prefix": "7e71db68c9a5422b"
+        "sha256_prefix": "b3b9f66f12b7c751"
     },
     "encode_write_kernel": {
         "bytes_per_symbol": 2.0506,
         "source": "encode.cu",
-        "sha256_prefix": "6bc7d2cb30f5e965"
+        "sha256_prefix": "95589fd6b6693e1e"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0056,
         "source": "histogram.cu",
-        "sha256_prefix": "19a0a2a5457d1407"
+        "sha256_prefix": "e6dfb9a64a2cdda3"
     },
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0001,
         "source": "build_tables.cu",
-        "sha256_prefix": "4da24da9e6f46b0d"
+        "sha256_prefix": "fec74e8b50068857"
     },
     "encode_compact_kernel": {
         "bytes_per_symbol": 1.7817,
         "source": "encode.cu",
-        "sha256_prefix": "6bc7d2cb30f5e965"
+        "sha256_prefix": "95589fd6b6693e1e"
     }
 }
 
 
+def source_digest(path):
+    """sha256 prefix of a CUDA source with comments and blank lines removed, so that editing a
+    comment does not invalidate a capture of the kernel."""
+    import hashlib
+    import re
+
+    txt = open(path).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    txt = re.sub(r"//[^\n]*", "", txt)
+    txt = "\n".join(ln.strip() for ln in txt.splitlines() if ln.strip())
+    return hashlib.sha256(txt.encode()).hexdigest()[:16]
+
+
 def measured_traffic(kernels, n_symbols):
     """Total DRAM bytes of the given kernels for n_symbols, or None if any capture is stale."""
-    import hashlib
-
     total = 0.0
     for k in kernels:
         m = MEASURED_TRAFFIC[k]
-        path = os.path.join(ROOT, "entropy_coded_lossless_b200", "csrc", m["source"])
-        if hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] != m["sha256_prefix"]:
+        if source_digest(os.path.join(ROOT, "entropy_coded_lossless_b200", "csrc", m["source"])) != m["sha256_prefix"]:
             return None
         total += m["bytes_per_symbol"] * n_symbols
     return total

@@ -4,7 +4,7 @@
 // DP C[i,k] = min_{j<i} { C[j,k-1] + Cost(j,i-1) } with backtracking from C[256,K]; derive the
 // per-range parameters (base, offset bits, encTable start, normalisation bias), rangeId[256], and an
 // L-entry tANS table from the range probabilities. The exact integer rules (fixed-point log2, cost,
-// tie-breaks, state-count allocation, spread) are FORMAT.md §2-§5; this kernel must reproduce them
+// tie-breaks, state-count allocation, spread) are SHN1 format §2-§5; this kernel must reproduce them
 // bit for bit, so it uses only integer arithmetic.
 //
 // Work is tiny (O(K·256²/2) min-plus steps per table) and latency-bound; one block of 512 threads
@@ -34,7 +34,7 @@ struct BuildShared {
   long long cost;
 };
 
-// Greedy state allocation on one warp (FORMAT.md §4): every range with a count starts with one
+// Greedy state allocation on one warp (SHN1 format §4): every range with a count starts with one
 // state; each further state goes to the range with the largest N_k * (LG(f_k + 1) - LG(f_k)),
 // ties to the smallest k. kPer ranges per lane (K <= 32 * kPer).
 template <int kPer>
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
     return;
   }
 
-  // ---- range selection (FORMAT.md §3) ---------------------------------------------------------
+  // ---- range selection (SHN1 format §3) ---------------------------------------------------------
   if (K == 256) {
     if (tid < 256) {
       S.lo[tid] = tid;
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   if (tid < 256) S.f[tid] = 0;
   __syncthreads();
 
-  // ---- state counts (FORMAT.md §4): one warp, greedy with smallest-k tie-break ---------------
+  // ---- state counts (SHN1 format §4): one warp, greedy with smallest-k tie-break ---------------
   if (tid < 32) {
     if (K <= 32) normalize_warp<1>(S, K, L, tid);
     else if (K <= 64) normalize_warp<2>(S, K, L, tid);
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   }
   __syncthreads();
 
-  // ---- spread (FORMAT.md §5) ------------------------------------------------------------------
+  // ---- spread (SHN1 format §5) ------------------------------------------------------------------
   const uint32_t step = (L >> 1) + (L >> 3) + 3;
   for (uint32_t t = tid; t < L; t += kBuildThreads) {
     int a = 0, b2 = K - 1;  // largest k with cumul[k] <= t

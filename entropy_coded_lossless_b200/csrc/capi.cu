@@ -87,7 +87,7 @@ size_t shn_table_bytes(const shn_params* p) { return params_ok(p) ? (size_t)SHN_
 size_t shn_encode_bound(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs) {
   uint64_t tc = 0;
   if (!params_ok(p) || !segs_ok(h_segs, n_segs, &tc, nullptr, p->chunk_symbols)) return 0;
-  // every chunk holds at most C symbols (FORMAT.md §6)
+  // every chunk holds at most C symbols (SHN1 format §6)
   const uint64_t words = tc * chunk_max_words(p->states_per_chunk, p->log2L, p->chunk_symbols);
   return (size_t)round_up(payload_offset(n_segs, p->K, tc) + 4 * words, 16);
 }

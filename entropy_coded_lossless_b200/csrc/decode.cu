@@ -2,7 +2,7 @@
 // gives the symbol s and the bit count; read the offset o and restore x = base[s] + o").
 //
 // Work layout. A persistent grid of 256-thread blocks walks tiles of 256 consecutive chunks; each
-// thread decodes one chunk of C symbols with S interleaved states (FORMAT.md §7), reading the chunk
+// thread decodes one chunk of C symbols with S interleaved states (SHN1 format §7), reading the chunk
 // backwards from its end sentinel.
 //
 // Tables. The decode table lives in shared memory as 8-byte entries
@@ -79,7 +79,7 @@ __device__ __forceinline__ DecHeader read_header(const uint8_t* c) {
 __device__ __forceinline__ uint32_t width_bits(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
 
 // Validates the header, then every segment descriptor and table record in parallel (each against its
-// successor), so later kernels may trust all offsets taken from them (FORMAT.md §6).
+// successor), so later kernels may trust all offsets taken from them (SHN1 format §6).
 __global__ void __launch_bounds__(256) decode_check_kernel(const uint8_t* __restrict__ comp, uint64_t comp_bytes,
                                                            shn_params p, DeviceStatus* st, uint64_t out_capacity) {
   __shared__ int s_ok;
@@ -166,7 +166,7 @@ __host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
   return l;
 }
 
-// Build decode tables (FORMAT.md §5) for segments seg0 .. seg0+nt-1. replicated: nt == 1, entry of
+// Build decode tables (SHN1 format §5) for segments seg0 .. seg0+nt-1. replicated: nt == 1, entry of
 // slot i, replica c at byte (i*16 + c)*8; plain: table t at t*L*8, entry i at +i*8. All threads of
 // the block take part; the caller synchronises before (readers of the old tables are done).
 __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, const SmemLayout& lay, uint32_t seg0,
@@ -265,14 +265,14 @@ struct ChunkCtx {
   uint64_t cb;          // chunk start, bytes from the stream start
   uint32_t nw;          // chunk words
   uint32_t tbase;       // shared-window address of slot 0's entry for this thread (replica / plain table)
-  uint64_t pos0;        // output position (symbols) of the chunk's first piece (FORMAT.md §6)
+  uint64_t pos0;        // output position (symbols) of the chunk's first piece (SHN1 format §6)
   uint32_t pos_stride;  // symbols between consecutive pieces of the chunk (16 * chunks in its group)
   uint32_t pieces;
   uint32_t last_len;    // symbols in the last piece (1..16)
 };
 
 // Output sinks: where a chunk's decoded symbols go. Pieces are 16 consecutive output positions
-// (FORMAT.md §6); put_pair/put receive raw bytes in their low 8 bits (junk above).
+// (SHN1 format §6); put_pair/put receive raw bytes in their low 8 bits (junk above).
 struct ByteSink {  // the INT8 tensor itself
   uint8_t* out;
   uint8_t* dst;

@@ -2,7 +2,7 @@
 //
 // Per value x (symbol u = x ^ 0x80): s = rangeId[u]; emit the offset u - base[s] in nb[s] bits;
 // emit the low state bits that renormalise X for s; move X through encTable (§4.2: table lookups,
-// shifts, masks and adds only). Chunks are independent (FORMAT.md §7): one thread encodes one chunk
+// shifts, masks and adds only). Chunks are independent (SHN1 format §7): one thread encodes one chunk
 // backwards with S interleaved states.
 //
 // The stream position of a chunk depends on the sizes of all chunks before it, so encoding runs
@@ -98,7 +98,7 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   cd.L = L;
 }
 
-// Run one chunk backwards (FORMAT.md §6-§7), calling sink(field, width) for every field. seg points
+// Run one chunk backwards (SHN1 format §6-§7), calling sink(field, width) for every field. seg points
 // at the segment's first byte; the chunk's symbols are its pieces in order, so the last piece is
 // coded first. Full pieces are 16-byte loads, which a warp's 32 chunks of one group issue as 512
 // consecutive bytes.
@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kScanBlock) scan_apply_kernel(const uint32_t* 
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) out[n] = sums[gridDim.x];
 }
 
-// ---- header, descriptors, table records, chunk index (FORMAT.md §6) -------------------------
+// ---- header, descriptors, table records, chunk index (SHN1 format §6) -------------------------
 __device__ __forceinline__ void st16(uint8_t* p, uint32_t v) {
   p[0] = (uint8_t)v;
   p[1] = (uint8_t)(v >> 8);

@@ -1,7 +1,7 @@
 // shn_internal.cuh — internal definitions shared by the libshn kernels and the C-ABI layer.
 //
-// The SHN1 stream layout and every table rule are those of FORMAT.md (the codec's bitstream
-// specification), which restates the Shannonic method ("Shannonic: Efficient Entropy-Optimal
+// The SHN1 stream layout and every table rule are those of the SHN1 format specification,
+// which restates the Shannonic method ("Shannonic: Efficient Entropy-Optimal
 // Compression for ML Workloads", MLSys 2026 notes, §4.1 preprocessing and §4.2 Algorithm 2).
 #pragma once
 
@@ -12,7 +12,7 @@
 
 namespace shn {
 
-// ---- stream layout (FORMAT.md §6) -------------------------------------------------------------
+// ---- stream layout (SHN1 format §6) -------------------------------------------------------------
 constexpr uint32_t kMagic = 0x314E4853u;  // "SHN1"
 constexpr uint32_t kHeaderBytes = 64;
 constexpr uint32_t kSegDescBytes = 32;
@@ -31,7 +31,7 @@ __host__ __device__ inline uint64_t chunk_max_words(uint32_t S, uint32_t R, uint
   return ((uint64_t)S * R + c * (uint64_t)(R + 8) + 1 + 31) / 32;
 }
 
-// ---- which symbols a chunk holds (FORMAT.md §6) -----------------------------------------------
+// ---- which symbols a chunk holds (SHN1 format §6) -----------------------------------------------
 // Chunks come in groups of up to 32; a group's symbols are cut into 16-symbol pieces dealt round
 // robin to its chunks. Chunk c of a segment of n symbols: group base symbol, index j in the group,
 // stride m (chunks in the group), number of pieces, and the length of its last piece (1..16).
@@ -131,7 +131,7 @@ __device__ __forceinline__ void report(DeviceStatus* st, uint32_t code, uint32_t
   if (atomicCAS(&st->status, 0u, code) == 0u) st->detail = detail;
 }
 
-// ---- FORMAT.md §2 fixed-point log2: 24 fraction bits by repeated squaring -------------------
+// ---- SHN1 format §2 fixed-point log2: 24 fraction bits by repeated squaring -------------------
 __device__ __forceinline__ uint32_t lg_fixed(uint32_t n) {
   if (n == 0) return 0;
   const int e = 31 - __clz(n);

@@ -4,7 +4,7 @@
  * The codec is the Shannonic scheme of "Shannonic: Efficient Entropy-Optimal Compression for ML
  * Workloads" (MLSys 2026 talk notes): a 256-bin histogram, a dynamic-programming split of the value
  * space into K contiguous ranges, and tANS over the range indices with raw fixed-width offsets
- * (§4, §4.1, §4.2 Algorithm 2). The bitstream ("SHN1") is fixed by FORMAT.md.
+ * (§4, §4.1, §4.2 Algorithm 2). The bitstream ("SHN1") is fixed by its own format specification.
  *
  * Conventions for every entry point:
  *  - Pointers named d_* are CUDA device pointers, h_* are host pointers. All memory belongs to the
@@ -53,7 +53,7 @@ typedef struct shn_segment {
   uint64_t length; /* number of INT8 values; must be < 2^32 */
 } shn_segment;
 
-/* Codec parameters (FORMAT.md §6 constraints). */
+/* Codec parameters (SHN1 format §6 constraints). */
 typedef struct shn_params {
   uint32_t K;                /* number of ranges, 1 <= K <= min(256, L); K = 256 is plain tANS */
   uint32_t log2L;            /* R: tANS state count L = 2^R, 4 <= R <= 12 */
@@ -71,7 +71,7 @@ typedef struct shn_table {
   uint32_t log2L;   /* R */
   uint32_t status;  /* SHN_OK, or SHN_ERR_INVALID_ARG when the histogram total is >= 2^32 */
   uint32_t w_max;   /* largest offset field width over the ranges */
-  int64_t dp_cost;  /* D[256][K] of the range DP, units of 2^-24 bit (FORMAT.md §3) */
+  int64_t dp_cost;  /* D[256][K] of the range DP, units of 2^-24 bit (SHN1 format §3) */
   uint64_t n;       /* histogram total */
   uint16_t f[256];  /* tANS state count of each range (sum = L); entries >= K are 0 */
   uint8_t lo[256];  /* first symbol u of each range; range k = [lo[k], lo[k+1]) with lo[K] = 256 */
@@ -83,7 +83,7 @@ typedef struct shn_table {
 uint32_t shn_version(void);
 const char* shn_status_string(int status);
 
-/* SHN_OK if p satisfies the FORMAT.md §6 constraints, else SHN_ERR_INVALID_ARG. */
+/* SHN_OK if p satisfies the SHN1 format §6 constraints, else SHN_ERR_INVALID_ARG. */
 int shn_check_params(const shn_params* p);
 
 /* Bytes of one table record in d_tables (constant, = sizeof(shn_table)). */
@@ -124,7 +124,7 @@ int shn_histogram(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_seg
  * Range selection and tANS tables for each histogram (Shannonic §4.1: DP range selection
  * C[i,k] = min_{j<i} C[j,k-1] + Cost(j,i-1) with backtracking from C[256,K]; per-range base,
  * offset width, encTable start and bias; rangeId[256]; an L-state tANS table from the range
- * probabilities). Exact rules: FORMAT.md §2-§5. One CUDA block per table.
+ * probabilities). Exact rules: SHN1 format §2-§5. One CUDA block per table.
  *  d_hist    device, n_tables*256 uint64 (as written by shn_histogram).
  *  d_tables  device, n_tables*shn_table_bytes(p) bytes, 256-byte aligned; fully overwritten.
  * A histogram whose total is >= 2^32 gets status SHN_ERR_INVALID_ARG in its record (and makes

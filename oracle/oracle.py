@@ -2,7 +2,7 @@
 
 Functions follow "Shannonic: Efficient Entropy-Optimal Compression for ML Workloads" (MLSys 2026
 talk notes) §4.1 (histogram, DP range selection, tables) and §4.2 (Algorithm 2), with every open
-detail fixed by FORMAT.md. Arrays are numpy; nothing here touches a GPU.
+detail fixed by the SHN1 format specification. Arrays are numpy; nothing here touches a GPU.
 """
 import ctypes
 import os
@@ -108,7 +108,7 @@ def _u8(x):
 
 
 def lg(n: int) -> int:
-    """FORMAT.md §2 fixed-point log2 (24 fraction bits)."""
+    """SHN1 format §2 fixed-point log2 (24 fraction bits)."""
     return int(lib().orc_lg(int(n)))
 
 

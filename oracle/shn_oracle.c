@@ -12,8 +12,8 @@
  *   §4.2  Algorithm 2: encode = rangeId, emit offset in nb[s] bits, emit normalisation bits,
  *         encTable transition; decode = decTable[X] gives the range and bit count, read offset,
  *         x = base[s] + o.
- * Every step the notes leave open is fixed by FORMAT.md (the SHN1 specification); the section
- * of FORMAT.md is named beside each function.
+ * Every step the notes leave open is fixed by the SHN1 format specification; its section
+ * is named beside each function.
  *
  * Plain C99 + pthreads (threads only split independent chunks / segments).
  */
@@ -44,7 +44,7 @@ static int ceil_log2_u32(uint32_t m) { /* smallest w with 2^w >= m, m >= 1 */
 static uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 /* ------------------------------------------------------------------------------------------ */
-/* FORMAT.md §2 — fixed-point log2 by repeated squaring of the normalised mantissa.            */
+/* SHN1 format §2 — fixed-point log2 by repeated squaring of the normalised mantissa.            */
 
 int64_t orc_lg(uint64_t n) {
   if (n == 0) return 0;
@@ -63,7 +63,7 @@ int64_t orc_lg(uint64_t n) {
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* §4.1 histogram h[x] over the symbols u = byte ^ 0x80 (FORMAT.md §1).                        */
+/* §4.1 histogram h[x] over the symbols u = byte ^ 0x80 (SHN1 format §1).                        */
 
 void orc_histogram(const uint8_t* bytes, uint64_t n, uint64_t hist[256]) {
   for (int u = 0; u < 256; u++) hist[u] = 0;
@@ -71,7 +71,7 @@ void orc_histogram(const uint8_t* bytes, uint64_t n, uint64_t hist[256]) {
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* §4.1 DP range selection (FORMAT.md §3). Generic alphabet size A <= 256 so that the tests can
+/* §4.1 DP range selection (SHN1 format §3). Generic alphabet size A <= 256 so that the tests can
  * compare it with a brute force over all partitions of small alphabets.                       */
 
 int orc_partition(const uint64_t* hist, int A, int K, uint16_t* lo, int64_t* cost_out) {
@@ -143,7 +143,7 @@ int orc_partition(const uint64_t* hist, int A, int K, uint16_t* lo, int64_t* cos
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* §4.1 "tANS table from the range probabilities p_k = N_k/N": state counts (FORMAT.md §4).
+/* §4.1 "tANS table from the range probabilities p_k = N_k/N": state counts (SHN1 format §4).
  * Greedy: every occupied range gets one state, then each remaining state goes to the largest
  * marginal gain N_k * (LG(f_k+1) - LG(f_k)); ties to the smallest k.                          */
 
@@ -181,7 +181,7 @@ int orc_normalize(const uint64_t* N, int K, int R, uint32_t* f) {
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* §4.1 per-range parameters and tANS tables (FORMAT.md §5).                                   */
+/* §4.1 per-range parameters and tANS tables (SHN1 format §5).                                   */
 
 int orc_tables_init(const uint16_t* lo, const uint32_t* f, int K, int R, orc_tables* t) {
   if (K < 1 || K > 256 || R < 4 || R > 12) return ORC_ERR_ARG;
@@ -248,7 +248,7 @@ int orc_build_segment_tables(const uint64_t hist[256], int K, int R, orc_tables*
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Bit strings, LSB-first (FORMAT.md §7).                                                       */
+/* Bit strings, LSB-first (SHN1 format §7).                                                       */
 
 typedef struct {
   uint32_t* words;
@@ -293,7 +293,7 @@ static uint32_t br_read(bitreader* br, int n) {
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* §4.2 Algorithm 2 for one chunk (FORMAT.md §7).                                              */
+/* §4.2 Algorithm 2 for one chunk (SHN1 format §7).                                              */
 
 static uint64_t chunk_max_words(int S, int R, uint64_t c) {
   return ((uint64_t)S * R + c * (uint64_t)(R + 8) + 1 + 31) / 32;
@@ -354,7 +354,7 @@ int orc_decode_chunk(const orc_tables* t, int S, const uint32_t* words, uint64_t
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Little-endian field access for the stream header (FORMAT.md §6).                            */
+/* Little-endian field access for the stream header (SHN1 format §6).                            */
 
 static void put16(uint8_t* p, uint16_t v) {
   p[0] = (uint8_t)v;
@@ -387,7 +387,7 @@ static int params_ok(const orc_params* p) {
 
 static uint64_t seg_chunks(uint64_t n, int C) { return (n + (uint64_t)C - 1) / (uint64_t)C; }
 
-/* FORMAT.md §6 "which symbols a chunk holds": chunks come in groups of up to 32; a group's symbols
+/* SHN1 format §6 "which symbols a chunk holds": chunks come in groups of up to 32; a group's symbols
  * are cut into 16-symbol pieces dealt round-robin to its chunks. Writes the positions (relative to
  * the segment start) of chunk c's symbols, in chunk order, to pos (if not NULL); returns the count. */
 static uint32_t chunk_positions(uint64_t n, int C, uint64_t c, uint64_t* pos) {
@@ -464,7 +464,7 @@ static void parallel_for(int n_threads, uint64_t n_items, void (*fn)(void*, uint
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Stream encoder (FORMAT.md §6–§7).                                                            */
+/* Stream encoder (SHN1 format §6–§7).                                                            */
 
 typedef struct {
   const uint8_t* input;
@@ -685,7 +685,7 @@ int orc_encode_stream_with_tables(const uint8_t* input, const orc_segment* segs,
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* Stream decoder (FORMAT.md §6–§7).                                                            */
+/* Stream decoder (SHN1 format §6–§7).                                                            */
 
 typedef struct {
   const uint8_t* stream;

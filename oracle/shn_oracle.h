@@ -8,7 +8,7 @@
  * Method: "Shannonic: Efficient Entropy-Optimal Compression for ML Workloads"
  * (MLSys 2026 talk notes) — §4.1 histogram, DP range selection, per-range parameters and tANS
  * tables; §4.2 Algorithm 2 encode/decode; §4 Theorem 1 (checked by the tests, not here).
- * Every detail the notes leave open follows FORMAT.md (the SHN1 stream specification).
+ * Every detail the notes leave open follows the SHN1 format specification.
  *
  * Parity pins: every function below is pinned by tests/test_oracle_*.py against brute force,
  * closed forms or the mathematics (see the header comment of each test file).
@@ -45,7 +45,7 @@ typedef struct {
   int32_t C; /* symbols per chunk */
 } orc_params;
 
-/* All tables of one segment (FORMAT.md §3–§5). */
+/* All tables of one segment (SHN1 format §3–§5). */
 typedef struct {
   int32_t K, R, L;
   uint16_t lo[257];         /* range k = [lo[k], lo[k+1]), lo[K] = 256 */
@@ -77,14 +77,14 @@ int orc_normalize(const uint64_t* N, int K, int R, uint32_t* f);
 int orc_tables_init(const uint16_t* lo, const uint32_t* f, int K, int R, orc_tables* t);
 int orc_build_segment_tables(const uint64_t hist[256], int K, int R, orc_tables* t, int64_t* dp_cost);
 
-/* One chunk, given its symbol sequence (FORMAT.md §6 says which tensor positions a chunk holds).
+/* One chunk, given its symbol sequence (SHN1 format §6 says which tensor positions a chunk holds).
  * Symbols are u = byte ^ 0x80. Returns words written, or -(error). */
 int64_t orc_encode_chunk(const orc_tables* t, int S, const uint8_t* bytes, uint32_t c, uint32_t* words,
                          uint64_t cap_words, uint64_t* payload_bits);
 int orc_decode_chunk(const orc_tables* t, int S, const uint32_t* words, uint64_t nwords, uint32_t c,
                      uint8_t* bytes);
 
-/* Whole SHN1 streams (FORMAT.md §6). */
+/* Whole SHN1 streams (SHN1 format §6). */
 uint64_t orc_stream_bound(const orc_params* p, const orc_segment* segs, int n_segs);
 int orc_encode_stream(const uint8_t* input, const orc_segment* segs, int n_segs, const orc_params* p,
                       int n_threads, uint8_t* out, uint64_t cap, uint64_t* out_bytes, orc_segment_stats* stats);

@@ -1,7 +1,7 @@
-"""Independent pure-Python reading of FORMAT.md (SHN1) and the paper's rate formulas, for tests.
+"""Independent pure-Python reading of the SHN1 format specification and the paper's rate formulas, for tests.
 
 Nothing here imports the oracle or the CUDA binding. It is a second, deliberately naive
-implementation of the stream layout (FORMAT.md §6), the tables (§5) and the decoder (§7), used on
+implementation of the stream layout (SHN1 format §6), the tables (§5) and the decoder (§7), used on
 small inputs to pin the oracle's bit order and field layout, plus fp64 helpers for the rate
 measurements of "Shannonic: Efficient Entropy-Optimal Compression for ML Workloads" (§4 Theorem 1,
 §5 %diff).
@@ -36,7 +36,7 @@ def parse_stream(buf):
 
 
 def chunk_positions(n, C, c):
-    """FORMAT.md §6: positions (relative to the segment start) of chunk c's symbols, in order."""
+    """SHN1 format §6: positions (relative to the segment start) of chunk c's symbols, in order."""
     nch = -(-n // C)
     grp, j = divmod(c, 32)
     m = min(32, nch - 32 * grp)
@@ -61,7 +61,7 @@ def chunk_words(st, seg_id, c):
 
 
 def spec_tables(lo, f, R):
-    """FORMAT.md §5 written out directly: spread, decode rows (sym, nb, next) and encode rows."""
+    """SHN1 format §5 written out directly: spread, decode rows (sym, nb, next) and encode rows."""
     L = 1 << R
     K = len(f)
     step = L // 2 + L // 8 + 3
@@ -88,7 +88,7 @@ def width_bits(lo, k):
 
 
 def spec_decode_chunk(words, lo, f, R, S, c):
-    """FORMAT.md §7 decoder, bit by bit. Returns (symbols u as a list, ok flag)."""
+    """SHN1 format §7 decoder, bit by bit. Returns (symbols u as a list, ok flag)."""
     L = 1 << R
     _, dec = spec_tables(lo, f, R)
     bits = []

@@ -1,5 +1,5 @@
 """The C-ABI library loads without a GPU and exports every entry point include/shn.h declares;
-host-only queries agree with the format (FORMAT.md §6) as the oracle computes it. No CUDA calls."""
+host-only queries agree with the format (SHN1 format §6) as the oracle computes it. No CUDA calls."""
 import os
 import re
 

@@ -7,7 +7,7 @@
   fixed-point log2           → bound against math.log2, exact at powers of two.
   §4.2 Algorithm 2           → round trip; K=1 (raw offsets, pins the bit order); forced uniform
                                table (every symbol exactly 4+4 bits); a single distinct value
-                               (0 payload bits); an independent bit-by-bit reader of FORMAT.md.
+                               (0 payload bits); an independent bit-by-bit reader of the SHN1 format.
   §4 Theorem 1               → rate closes to the closed form within 0.01 bit; the i.i.d. rate
                                matches the exact stationary rate of the tANS state chain.
   §4 Condition 3             → its sign predicts which of Shannonic / plain tANS is shorter.
@@ -191,7 +191,7 @@ def test_tables_structure_and_inverse(orc):
             t = orc.tables(lo, f, R)
             spread = np.array(t.spread[:L])
             assert (np.bincount(spread, minlength=K)[:K] == f).all()
-            # the spread and decode rows equal an independent reading of FORMAT.md §5
+            # the spread and decode rows equal an independent reading of SHN1 format §5
             s_ref, dec_ref = spec.spec_tables([int(v) for v in lo], [int(v) for v in f], R)
             assert list(spread) == s_ref
             assert [(t.dec_sym[i], t.dec_nb[i], t.dec_next[i]) for i in range(L)] == dec_ref
@@ -281,7 +281,7 @@ def test_single_value_has_empty_payload(orc):
 
 
 def test_chunk_mapping_partitions_each_segment():
-    """FORMAT.md §6: the chunks of a segment hold every symbol exactly once, at most C each, and in
+    """SHN1 format §6: the chunks of a segment hold every symbol exactly once, at most C each, and in
     a full group of 32 the k-th pieces of the chunks are 512 consecutive symbols."""
     for n, C in [(0, 128), (1, 128), (128, 128), (129, 128), (5000, 256), (32 * 256, 256), (33 * 256 + 7, 256),
                  (70 * 1024 + 3, 1024), (1_000_003, 4096)]:
