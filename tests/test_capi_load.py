@@ -66,3 +66,39 @@ def test_encode_bound_matches_format(lib, orc, K, R, S, C):
 def test_oversized_segment_rejected(lib):
     p = shn.CodecParams()
     assert shn.encode_bound(p, [(0, 1 << 32)]) == 0
+
+
+def test_offload_queries_and_host_checks(lib, orc):
+    """Host-side logic of the offload entry points, no CUDA call: workspace query, and the checks
+    shn_decode_from_host makes on the host streams before it enqueues anything."""
+    import ctypes
+
+    import numpy as np
+
+    p = shn.CodecParams(16, 7, 4096, 4)
+    segs = [(0, 1 << 20), (1 << 20, 5000), (1 << 20 | 5000, 3 << 20)]
+    ends = [1, 3]
+    w = shn.offload_workspace_bytes(p, segs, ends)
+    # at least two staging streams of the larger batch and its single-pass encoder workspace
+    assert w >= 2 * shn.encode_bound(p, segs[1:]) + shn.encode_workspace_bytes(p, segs[1:])
+    assert shn.offload_workspace_bytes(p, segs, [2, 1]) == 0  # batch ends must not decrease
+
+    x = np.zeros(1000, np.int8)
+    stream, _ = orc.encode(x, K=16, R=7, S=4, C=4096)
+    L = shn.lib()
+    fake_dev = 1 << 20  # never dereferenced: every check below fails before a CUDA call
+
+    def call(buf, nbytes, out_cap, staging_bytes):
+        arr = np.ascontiguousarray(buf)
+        ptrs = (ctypes.c_void_p * 1)(arr.ctypes.data)
+        sizes = (ctypes.c_size_t * 1)(nbytes)
+        offs = (ctypes.c_size_t * 1)(0)
+        return L.shn_decode_from_host(ptrs, sizes, 1, ctypes.byref(p.c()), fake_dev, staging_bytes, fake_dev, 256,
+                                      fake_dev, offs, out_cap, None, None)
+
+    bad = stream.copy()
+    bad[0] ^= 0xFF
+    assert call(bad, stream.size, 1000, 1 << 20) == shn.SHN_ERR_CORRUPT
+    assert call(stream, 10, 1000, 1 << 20) == shn.SHN_ERR_CORRUPT  # shorter than a header
+    assert call(stream, stream.size, 999, 1 << 20) == shn.SHN_ERR_CAPACITY
+    assert call(stream, stream.size, 1000, stream.size) == shn.SHN_ERR_WORKSPACE  # room for one stream only
