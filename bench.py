@@ -39,8 +39,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="kv", choices=["kv", "weight", "sweep", "activations", "int4", "regen"],
-                    help="regen: time table regeneration (histogram + tables) only")
+    ap.add_argument("--workload", default="kv",
+                    choices=["kv", "weight", "sweep", "activations", "int4", "regen", "sweepgrid"],
+                    help="regen: time table regeneration only; sweepgrid: rate and time over the whole "
+                         "entropy x chunk x K x L grid of the 1 GiB sweep")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -350,6 +352,53 @@ def run_regen(args):
                       "cases": cases}), flush=True)
 
 
+def run_sweepgrid(args):
+    """Every point of the 1 GiB sweep (H x C x K x L, 108 points): payload and total bits/value
+    against the entropy, and the median encode/decode time of 3 runs (inputs > L2)."""
+    from entropy_coded_lossless_b200 import shn
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    pts, cur_h, x = [], None, None
+    for pt in inputs.sweep_points():
+        if pt["H"] != cur_h:
+            del x
+            torch.cuda.empty_cache()
+            x = inputs.sweep_stream_int8(pt["H"], seed=4, device=dev)
+            cur_h = pt["H"]
+        segs = [(0, x.numel())]
+        p_dict = dict(K=pt["K"], log2L=int(pt["L"]).bit_length() - 1, chunk_symbols=pt["C"], states_per_chunk=4)
+        p = shn.CodecParams(**p_dict)
+        codec = shn.Codec(segs, p, device=dev)
+        out = torch.empty(x.numel(), dtype=torch.uint8, device=dev)
+        codec.histogram(x)
+        codec.build()
+        te, td = [], []
+        for _ in range(3):
+            a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+            codec.encode(x)
+            b.record(stream)
+            codec.decode(codec.stream_buf, codec.stream_buf.numel(), out)
+            c.record(stream)
+            torch.cuda.synchronize()
+            te.append(a.elapsed_time(b))
+            td.append(b.elapsed_time(c))
+        ok = codec.status("enc")[0] == 0 and codec.status("dec")[0] == 0 and torch.equal(out, x.view(torch.uint8))
+        nbytes = int(codec.out_bytes.item())
+        rate = stream_rate(codec.stream_buf[:nbytes].cpu().numpy(), segs, p_dict, codec.hist.cpu().numpy())
+        pts.append({"H": pt["H"], "C": pt["C"], "K": pt["K"], "L": pt["L"], "payload": rate["payload"],
+                    "total": rate["total"], "entropy": rate["entropy"], "diff_pct": rate["diff_pct"],
+                    "encode_ms": statistics.median(te), "decode_ms": statistics.median(td), "correct": bool(ok)})
+        del codec, out
+    print(json.dumps({"metric": "bits/symbol vs H and codec time over the 1 GiB sweep grid", "value":
+                      sum(1 for q in pts if q["K"] == 16 and q["L"] == 128 and q["diff_pct"] <= 1.0),
+                      "unit": "points with K=16, L=128 within 1% of H", "n_gpus": 1, "higher_is_better": True,
+                      "dtype": "u8", "data": "synthetic", "config": {"workload": "sweepgrid"}, "points": pts}),
+          flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -405,6 +454,8 @@ def main():
         return run_reference(args)
     if args.workload == "regen":
         return run_regen(args)
+    if args.workload == "sweepgrid":
+        return run_sweepgrid(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
