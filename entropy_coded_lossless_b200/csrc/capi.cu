@@ -186,30 +186,36 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
   const shn_table* tables = static_cast<const shn_table*>(d_tables);
   if (cudaMemsetAsync(wb, 0, 8, s) != cudaSuccess) return SHN_ERR_CUDA;
 
-  // segment batches (kernel parameters), built once and reused by every pass
+  // Segment batches (kernel parameters), built once and reused by every pass. A batch holds
+  // consecutive segments (the header pass indexes a contiguous chunk range per batch) of one kind:
+  // segments of at most kEncSmallMaxChunks chunks are coded by one-warp blocks with unreplicated
+  // tables, the others by kEncBlockThreads-thread blocks with lane-replicated tables.
   std::vector<EncBatch> batches;
   {
-    uint64_t chunk = 0, out_off = 0;
-    for (uint32_t s0 = 0; s0 < n_segs; s0 += kSegBatch) {
-      batches.emplace_back();
-      EncBatch& b = batches.back();
-      memset(&b, 0, sizeof(b));
-      b.n = (n_segs - s0 < (uint32_t)kSegBatch) ? n_segs - s0 : (uint32_t)kSegBatch;
-      uint64_t blocks = 0;
-      for (uint32_t i = 0; i < b.n; ++i) {
-        const shn_segment& sg = h_segs[s0 + i];
-        b.offset[i] = sg.offset;
-        b.out_offset[i] = out_off;
-        b.length[i] = (uint32_t)sg.length;
-        b.first_chunk[i] = (uint32_t)chunk;
-        b.block_start[i] = (uint32_t)blocks;
-        b.seg_index[i] = s0 + i;
-        const uint64_t nc = n_chunks(sg.length, p->chunk_symbols);
-        blocks += (nc + kEncBlockThreads - 1) / kEncBlockThreads;
-        chunk += nc;
-        out_off += sg.length;
+    uint64_t chunk = 0, out_off = 0, blocks = 0;
+    for (uint32_t si = 0; si < n_segs; ++si) {
+      const shn_segment& sg = h_segs[si];
+      const uint64_t nc = n_chunks(sg.length, p->chunk_symbols);
+      const uint32_t small = (nc <= kEncSmallMaxChunks) ? 1u : 0u;
+      if (batches.empty() || batches.back().n == (uint32_t)kSegBatch || batches.back().small != small) {
+        batches.emplace_back();
+        memset(&batches.back(), 0, sizeof(EncBatch));
+        batches.back().small = small;
+        blocks = 0;
       }
+      EncBatch& b = batches.back();
+      const uint32_t i = b.n++;
+      b.offset[i] = sg.offset;
+      b.out_offset[i] = out_off;
+      b.length[i] = (uint32_t)sg.length;
+      b.first_chunk[i] = (uint32_t)chunk;
+      b.block_start[i] = (uint32_t)blocks;
+      b.seg_index[i] = si;
+      const uint64_t nt = small ? (uint64_t)kEncSmallThreads : (uint64_t)kEncBlockThreads;
+      blocks += (nc + nt - 1) / nt;
       b.total_blocks = (uint32_t)blocks;
+      chunk += nc;
+      out_off += sg.length;
     }
   }
   // single pass: code every chunk into its slot (recording sizes); two passes: count sizes first

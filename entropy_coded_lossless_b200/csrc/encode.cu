@@ -42,8 +42,8 @@ __host__ __device__ inline uint32_t enc_copies(uint32_t R) {
   while (c > 1 && (kEncSlot << R) * c > kEncCopyBudget) c >>= 1;
   return c;
 }
-__host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t R) {
-  return 256 * kSymCopies * 8 + (kEncSlot << R) * enc_copies(R);
+__host__ __device__ inline uint32_t enc_table_smem_bytes(uint32_t R, bool plain = false) {
+  return plain ? 256 * 8 + (kEncSlot << R) : 256 * kSymCopies * 8 + (kEncSlot << R) * enc_copies(R);
 }
 
 // Segment of this block: largest s with block_start[s] <= blockIdx.x.
@@ -59,8 +59,11 @@ __device__ __forceinline__ int block_segment(const EncBatch& b) {
 
 // Algorithm 2 per symbol, on the lane-interleaved tables. State X in [L, 2L). Addresses are 32-bit
 // shared-window addresses.
+// PLAIN: one copy of each table (small segments; lanes may conflict on a bank).
+template <bool PLAIN>
 struct Coder {
-  uint32_t sym;      // this lane's column of sym: + raw byte * 128
+  static constexpr uint32_t kSymRow = PLAIN ? 8u : kSymCopies * 8u;  // bytes per raw-byte row of sym
+  uint32_t sym;      // this lane's column of sym: + raw byte * kSymRow
   uint32_t enc;      // this lane's column of enc, biased by -4096 rows (the +4096 in .y's start field)
   uint32_t enc_row;  // bytes per enc index (2 * copies)
   uint32_t L;
@@ -68,7 +71,7 @@ struct Coder {
   // CHECK: accumulate .y into flags (bit 15 set for a byte absent from the table's histogram).
   template <bool CHECK>
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
-    const uint2 e = lds64(sym + b * (kSymCopies * 8));
+    const uint2 e = lds64(sym + b * kSymRow);
     const uint32_t nb = (X + e.x) >> 16;
     const uint32_t q = X >> nb;
     const uint32_t r = X - (q << nb);                   // the nb low state bits
@@ -80,18 +83,20 @@ struct Coder {
   }
 };
 
-__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t R, Coder& cd) {
+template <bool PLAIN>
+__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t R, Coder<PLAIN>& cd) {
   const uint32_t L = 1u << R;
-  const uint32_t copies = enc_copies(R);
+  const uint32_t copies = PLAIN ? 1u : enc_copies(R);
+  const uint32_t sym_copies = PLAIN ? 1u : kSymCopies;
   const uint2* sym = table_sym(t);
   const uint16_t* enc = table_enc(t);
   uint2* s2 = reinterpret_cast<uint2*>(smem);
-  unsigned char* e2 = smem + 256 * kSymCopies * 8;
-  for (uint32_t i = threadIdx.x; i < 256 * kSymCopies; i += blockDim.x) s2[i] = sym[i / kSymCopies];
+  unsigned char* e2 = smem + 256 * sym_copies * 8;
+  for (uint32_t i = threadIdx.x; i < 256 * sym_copies; i += blockDim.x) s2[i] = sym[i / sym_copies];
   for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x)
     *reinterpret_cast<uint16_t*>(e2 + i * kEncSlot) = enc[i / copies];
   const uint32_t lane = threadIdx.x & 31;
-  cd.sym = smem_addr(smem) + (lane & (kSymCopies - 1)) * 8;
+  cd.sym = smem_addr(smem) + (lane & (sym_copies - 1)) * 8;
   cd.enc_row = kEncSlot * copies;
   // entry e of copy c is at e2 + (e * copies + c) * kEncSlot
   cd.enc = smem_addr(e2) + (lane & (copies - 1)) * kEncSlot - 4096u * cd.enc_row;
@@ -102,8 +107,8 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
 // at the segment's first byte; the chunk's symbols are its pieces in order, so the last piece is
 // coded first. Full pieces are 16-byte loads, which a warp's 32 chunks of one group issue as 512
 // consecutive bytes.
-template <int S, bool PAIRS, bool CHECK, class Sink>
-__device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, const ChunkGeo& g, uint32_t* st,
+template <int S, bool PAIRS, bool CHECK, class CoderT, class Sink>
+__device__ __forceinline__ void code_chunk(const CoderT& cd, const uint8_t* seg, const ChunkGeo& g, uint32_t* st,
                                            uint32_t& flags, Sink& sink) {
   int k = (int)g.pieces - 1;
   if (g.last_len < 16) {  // the group's short last piece, symbol by symbol
@@ -115,7 +120,7 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
       for (int z = 1; z < S; ++z)
         if (z == q) x = st[z];
       uint32_t w;
-      const uint32_t field = cd.step<CHECK>(src[t], x, w, flags);
+      const uint32_t field = cd.template step<CHECK>(src[t], x, w, flags);
 #pragma unroll
       for (int z = 0; z < S; ++z)
         if (z == q) st[z] = x;
@@ -145,8 +150,8 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
         const uint32_t b1 = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
         const uint32_t b2 = __byte_perm(wv[(r - 1) >> 2], 0u, 0x4440u + (uint32_t)((r - 1) & 3));
         uint32_t w1, w2;
-        const uint32_t f1 = cd.step<CHECK>(b1, st[r & (S - 1)], w1, flags);
-        const uint32_t f2 = cd.step<CHECK>(b2, st[(r - 1) & (S - 1)], w2, flags);
+        const uint32_t f1 = cd.template step<CHECK>(b1, st[r & (S - 1)], w1, flags);
+        const uint32_t f2 = cd.template step<CHECK>(b2, st[(r - 1) & (S - 1)], w2, flags);
         sink(f1 | (f2 << w1), w1 + w2);
       }
     } else {
@@ -154,7 +159,7 @@ __device__ __forceinline__ void code_chunk(const Coder& cd, const uint8_t* seg, 
       for (int r = 15; r >= 0; --r) {
         const uint32_t b = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
         uint32_t w;
-        const uint32_t field = cd.step<CHECK>(b, st[r & (S - 1)], w, flags);
+        const uint32_t field = cd.template step<CHECK>(b, st[r & (S - 1)], w, flags);
         sink(field, w);
       }
     }
@@ -227,18 +232,19 @@ struct RingWriter {
   }
 };
 
-template <int S, bool PAIRS>
-__global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t* __restrict__ in,
-                                                                   const __grid_constant__ EncBatch b,
-                                                                   const shn_table* __restrict__ tables,
-                                                                   const EncodeLayout lay, EncodeWork w) {
+// SMALL: kEncSmallThreads-thread blocks with unreplicated tables (segments of few chunks).
+template <int S, bool PAIRS, bool SMALL>
+__global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode_sizes_kernel(
+    const uint8_t* __restrict__ in, const __grid_constant__ EncBatch b, const shn_table* __restrict__ tables,
+    const EncodeLayout lay, EncodeWork w) {
+  constexpr int NT = SMALL ? kEncSmallThreads : kEncThreads;
   extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  Coder cd;
+  Coder<SMALL> cd;
   load_coder(esm, t, lay.R, cd);
   __syncthreads();
-  const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
+  const uint32_t c = (blockIdx.x - b.block_start[seg]) * NT + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
@@ -257,26 +263,25 @@ __global__ void __launch_bounds__(kEncThreads) encode_sizes_kernel(const uint8_t
 // stream, from the word offsets of the scan. Single-pass mode (SLOTS = true): into the chunk's own
 // worst-case-size slot in the workspace, recording the word count (and, as the size pass would,
 // flagging symbols absent from the table); encode_compact_kernel then moves the slots into place.
-template <int S, bool PAIRS, bool SLOTS>
-__global__ void __launch_bounds__(kEncThreads) encode_write_kernel(const uint8_t* __restrict__ in,
-                                                                   const __grid_constant__ EncBatch b,
-                                                                   const shn_table* __restrict__ tables,
-                                                                   const EncodeLayout lay, EncodeWork w,
-                                                                   uint8_t* __restrict__ out) {
+template <int S, bool PAIRS, bool SLOTS, bool SMALL>
+__global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode_write_kernel(
+    const uint8_t* __restrict__ in, const __grid_constant__ EncBatch b, const shn_table* __restrict__ tables,
+    const EncodeLayout lay, EncodeWork w, uint8_t* __restrict__ out) {
+  constexpr int NT = SMALL ? kEncSmallThreads : kEncThreads;
   if (*(volatile uint32_t*)&w.status->status != 0) return;
   extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
-  Coder cd;
+  Coder<SMALL> cd;
   load_coder(esm, t, lay.R, cd);
   __syncthreads();
-  const uint32_t c = (blockIdx.x - b.block_start[seg]) * kEncThreads + threadIdx.x;
+  const uint32_t c = (blockIdx.x - b.block_start[seg]) * NT + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
   const ChunkGeo geo = chunk_geo(len_seg, lay.C, c);
   const uint64_t g = (uint64_t)b.first_chunk[seg] + c;
   RingWriter rw;
-  rw.ring = smem_addr(esm) + (uint32_t)round_up(enc_table_smem_bytes(lay.R), 16) + threadIdx.x * (kRingStride * 4);
+  rw.ring = smem_addr(esm) + (uint32_t)round_up(enc_table_smem_bytes(lay.R, SMALL), 16) + threadIdx.x * (kRingStride * 4);
   if (SLOTS) {
     rw.payload = w.slots + g * w.slot_words;
     rw.wp = rw.fp = 0;
@@ -515,25 +520,40 @@ __global__ void encode_header_kernel(const __grid_constant__ EncBatch b, const s
   st32(out + lay.index_offset + 4 * g, (uint32_t)(w.word_offset[g] - w.word_offset[b.first_chunk[lo]]));
 }
 
+template <int S, bool PAIRS, bool SMALL>
+static cudaError_t launch_sizes_small_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
+                                        const EncodeLayout& lay, const EncodeWork& w, cudaStream_t s) {
+  const size_t smem = enc_table_smem_bytes(lay.R, SMALL);
+  cudaError_t e = cudaFuncSetAttribute(encode_sizes_kernel<S, PAIRS, SMALL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  encode_sizes_kernel<S, PAIRS, SMALL><<<b.total_blocks, SMALL ? kEncSmallThreads : kEncThreads, smem, s>>>(
+      d_in, b, d_tables, lay, w);
+  return cudaGetLastError();
+}
 template <int S, bool PAIRS>
 static cudaError_t launch_sizes_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, cudaStream_t s) {
-  const size_t smem = enc_table_smem_bytes(lay.R);
-  cudaError_t e = cudaFuncSetAttribute(encode_sizes_kernel<S, PAIRS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  return b.small ? launch_sizes_small_t<S, PAIRS, true>(d_in, b, d_tables, lay, w, s)
+                 : launch_sizes_small_t<S, PAIRS, false>(d_in, b, d_tables, lay, w, s);
+}
+template <int S, bool PAIRS, bool SLOTS, bool SMALL>
+static cudaError_t launch_write_small_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
+                                        const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out,
+                                        cudaStream_t s) {
+  constexpr int NT = SMALL ? kEncSmallThreads : kEncThreads;
+  const size_t smem = round_up(enc_table_smem_bytes(lay.R, SMALL), 16) + NT * kRingStride * 4;
+  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, PAIRS, SLOTS, SMALL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  encode_sizes_kernel<S, PAIRS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w);
+  encode_write_kernel<S, PAIRS, SLOTS, SMALL><<<b.total_blocks, NT, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
   return cudaGetLastError();
 }
 template <int S, bool PAIRS, bool SLOTS>
 static cudaError_t launch_write_t(const uint8_t* d_in, const EncBatch& b, const shn_table* d_tables,
                                   const EncodeLayout& lay, const EncodeWork& w, uint8_t* d_out, cudaStream_t s) {
-  const size_t smem = round_up(enc_table_smem_bytes(lay.R), 16) + kEncThreads * kRingStride * 4;
-  cudaError_t e = cudaFuncSetAttribute(encode_write_kernel<S, PAIRS, SLOTS>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  encode_write_kernel<S, PAIRS, SLOTS><<<b.total_blocks, kEncThreads, smem, s>>>(d_in, b, d_tables, lay, w, d_out);
-  return cudaGetLastError();
+  return b.small ? launch_write_small_t<S, PAIRS, SLOTS, true>(d_in, b, d_tables, lay, w, d_out, s)
+                 : launch_write_small_t<S, PAIRS, SLOTS, false>(d_in, b, d_tables, lay, w, d_out, s);
 }
 
 // Two fields fit one 32-bit append when they are <= 16 bits each, i.e. L <= 256.

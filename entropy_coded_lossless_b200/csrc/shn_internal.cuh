@@ -91,6 +91,10 @@ inline int sm_count_for_launch() {
 #define ENC_THREADS 256
 #endif
 constexpr int kEncBlockThreads = ENC_THREADS;
+// Segments of at most kEncSmallMaxChunks chunks are coded by one-warp blocks with unreplicated
+// tables (a few KB of shared memory), so that many small tensors share an SM.
+constexpr int kEncSmallThreads = 32;
+constexpr uint32_t kEncSmallMaxChunks = 64;
 
 // ---- shared-memory accesses by 32-bit shared-window address ------------------------------------
 // The per-symbol loops address their tables and rings with 32-bit shared addresses (no 64-bit
@@ -163,6 +167,7 @@ struct HistBatch {
 struct EncBatch {
   uint32_t n;
   uint32_t total_blocks;
+  uint32_t small;                  // 1: kEncSmallThreads-thread blocks, unreplicated tables
   uint64_t offset[kSegBatch];      // byte offset in d_in
   uint64_t out_offset[kSegBatch];  // sum of the lengths of all earlier segments
   uint32_t length[kSegBatch];
