@@ -124,9 +124,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "b3b9f66f12b7c751"
     },
     "encode_write_kernel": {
-        "bytes_per_symbol": 2.0506,
+        "bytes_per_symbol": 2.0516,
         "source": "encode.cu",
-        "sha256_prefix": "95589fd6b6693e1e"
+        "sha256_prefix": "bfd8deb88df791ab"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0056,
@@ -139,9 +139,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "fec74e8b50068857"
     },
     "encode_compact_kernel": {
-        "bytes_per_symbol": 1.7817,
+        "bytes_per_symbol": 1.782,
         "source": "encode.cu",
-        "sha256_prefix": "95589fd6b6693e1e"
+        "sha256_prefix": "bfd8deb88df791ab"
     }
 }
 
