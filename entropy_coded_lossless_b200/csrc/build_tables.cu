@@ -17,6 +17,18 @@
 namespace shn {
 
 constexpr int kBuildThreads = 512;
+
+// LG(c) for every c < 2^17, filled by lg_table_kernel on the launching stream before a build of
+// many tables (more than one wave of blocks); tables whose segment total is below 2^17 then look
+// LG up instead of running the 24 squaring steps per range. Values are those of lg_fixed.
+constexpr uint32_t kLgTableSize = 1u << 17;
+constexpr uint32_t kLgTableMinTables = 256;  // builds of fewer tables compute LG directly
+__device__ uint32_t g_lg_table[kLgTableSize];
+
+__global__ void __launch_bounds__(256) lg_table_kernel() {
+  for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < kLgTableSize; c += gridDim.x * blockDim.x)
+    g_lg_table[c] = lg_fixed(c);
+}
 constexpr int kPairs = 256 * 257 / 2;  // ranges [j, i), 0 <= j < i <= 256
 
 __device__ __forceinline__ uint32_t ceil_log2_width(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
@@ -95,7 +107,8 @@ __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L
 }
 
 __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsigned long long* __restrict__ hist_all,
-                                                                     shn_params p, shn_table* __restrict__ tables_out) {
+                                                                     shn_params p, shn_table* __restrict__ tables_out,
+                                                                     uint32_t use_lg_table) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BuildShared& S = *reinterpret_cast<BuildShared*>(smem_raw);
   uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));          // kPairs cost factors
@@ -156,11 +169,13 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   } else {
     // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30; warp w
     // fills the rows i = w+1, w+17, ... (about the same number of pairs per warp)
+    const bool lookup = use_lg_table && S.pre[256] < kLgTableSize;  // every count of the segment is < 2^17
     for (int i = 1 + (tid >> 5); i <= 256; i += kBuildThreads / 32) {
       const uint32_t pi = S.pre[i];
       uint32_t* row = lgc + i * (i - 1) / 2;
       for (int j = tid & 31; j < i; j += 32)
-        row[j] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) - (int32_t)lg_fixed(pi - S.pre[j]));
+        row[j] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) -
+                            (int32_t)(lookup ? __ldg(g_lg_table + (pi - S.pre[j])) : lg_fixed(pi - S.pre[j])));
     }
     for (int i = tid; i <= 256; i += kBuildThreads) S.drow[0][i] = (i == 0) ? 0 : LLONG_MAX;
     __syncthreads();
@@ -326,8 +341,13 @@ cudaError_t launch_build_tables(const uint64_t* d_hist, uint32_t n_tables, const
   const size_t smem = sizeof(BuildShared) + sizeof(uint32_t) * kPairs + (size_t)p.K * 257;
   cudaError_t e = cudaFuncSetAttribute(build_tables_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const uint32_t use_table = n_tables >= kLgTableMinTables ? 1u : 0u;
+  if (use_table) {
+    lg_table_kernel<<<128, 256, 0, s>>>();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   build_tables_kernel<<<n_tables, kBuildThreads, smem, s>>>(reinterpret_cast<const unsigned long long*>(d_hist), p,
-                                                            d_tables);
+                                                            d_tables, use_table);
   return cudaGetLastError();
 }
 
