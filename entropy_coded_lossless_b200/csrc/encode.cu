@@ -5,18 +5,22 @@
 // shifts, masks and adds only). Chunks are independent (SHN1 format §7): one thread encodes one chunk
 // backwards with S interleaved states.
 //
-// The stream position of a chunk depends on the sizes of all chunks before it, so encoding runs
-// in passes: (1) every thread runs its chunk's state machine and records the chunk's word count,
-// (2) an exclusive scan turns counts into word offsets, (3) the header, segment descriptors, table
-// records and chunk index are written, (4) every thread re-runs its chunk and writes the words to
-// their final place. No device-wide spin waits; everything is ordered by the stream.
+// The stream position of a chunk depends on the sizes of all chunks before it. With a workspace
+// large enough for one worst-case slot per chunk the state machine runs once: (1) every thread codes
+// its chunk into its slot and records the word count, (2) an exclusive scan turns counts into word
+// offsets, (3) the header, segment descriptors, table records and chunk index are written, (4) one
+// warp per chunk moves the slot to its final place. With the minimal workspace it runs twice:
+// (1) counts only, (2), (3), then (4) every thread re-runs its chunk and writes the words in place.
+// No device-wide spin waits; everything is ordered by the stream.
 //
 // Shared-memory tables. Each block codes chunks of one segment and keeps Algorithm 2's per-range
-// form in shared memory: sym[raw byte] = {bias, (start + 4096) | offset << 16 | w << 24 | absent << 31}
-// and enc[L] (next state). A warp's 32 lookups use 32 unrelated indices, so both tables are stored
-// lane-interleaved: sym 16 times ([byte][16] x 8 bytes: an 8-byte load is served per half-warp, so
-// the 16 lanes of a phase always hit 16 distinct bank pairs) and enc up to 32 times ([index][copies]
-// x 2 bytes: every lane reads its own bank). Lookups are conflict-free whatever the data.
+// form in shared memory: sym[raw byte] = {bias, offset | w << 8 | (start + 4096) << 16}, with
+// bit 15 marking a byte absent from the table's histogram, and enc[L] (next state). A warp's 32
+// lookups use 32 unrelated indices, so both tables are stored lane-interleaved: sym 16 times
+// ([byte][16] x 8 bytes: an 8-byte load is served per half-warp, so the 16 lanes of a phase always
+// hit 16 distinct bank pairs) and enc up to 32 times ([index][copies] x 4-byte slots: every lane
+// reads its own bank). Lookups are conflict-free whatever the data. Segments of at most 64 chunks
+// use one-warp blocks and a single copy of each table instead (small tensors, many per SM).
 #include "shn_internal.cuh"
 
 namespace shn {
