@@ -20,8 +20,10 @@
 //
 // Bits. Each thread keeps a 64-bit window (two words) of its chunk in registers and refills it from
 // a private 128-byte ring in shared memory, which cp.async (16-byte, L2-only) copies fill ahead of
-// use. All shared-memory accesses of the per-symbol loop use 32-bit shared-window addresses. Two symbols are extracted per window position (fields are <= 16 bits for L <= 256). Decoded
-// bytes go out as 16-byte stores.
+// use. All shared-memory accesses of the per-symbol loop use 32-bit shared-window addresses. Two
+// symbols are extracted per window position when fields are <= 16 bits (L <= 256), one otherwise
+// (fields <= 20 bits, L <= 4096). Decoded values go to an output sink: the INT8 tensor (16-byte
+// stores of 16 values) or, fused with the consumer, bf16 values dequantised by a per-group scale.
 //
 // Robustness. Corrupt input never causes an out-of-bounds access: descriptors and the chunk index
 // are validated against the stream and output sizes, the ring is filled only from the thread's own
