@@ -478,9 +478,17 @@ def main():
     stream = torch.cuda.current_stream()
     comp_cap = codec.stream_buf.numel()
     if args.profile_only:
+        # (kv: also the fused bf16 decode after each INT8 decode, so its launches can be captured too)
+        scales = y16 = None
+        if args.workload == "kv":
+            scales = torch.cat([inputs.kv_cache_segment_int8_and_scales(i // 2, i % 2, seed=2 + rank, device=dev)[1]
+                                for i in range(len(segs))])
+            y16 = torch.empty(n, dtype=torch.bfloat16, device=dev)
         for _ in range(2):
             codec.compress(x)
             codec.decode(codec.stream_buf, comp_cap, out)
+            if y16 is not None:
+                shn.shn_decode_bf16(codec.stream_buf, comp_cap, p, scales, 7, codec.work_dec, y16)
         torch.cuda.synchronize()
         ok = codec.status("enc")[0] == 0 and codec.status("dec")[0] == 0 and torch.equal(out, x.view(torch.uint8))
         print(json.dumps({"profile_case": desc, "symbols": n, "stream_bytes": int(codec.out_bytes.item()),
