@@ -119,7 +119,7 @@ def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
 # is stale and the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     "decode_kernel": {
-        "bytes_per_symbol": 1.8894,
+        "bytes_per_symbol": 1.8881,
         "source": "decode.cu",
         "sha256_prefix": "b3b9f66f12b7c751"
     },
