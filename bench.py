@@ -119,14 +119,14 @@ def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
 # is stale and the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     "decode_kernel": {
-        "bytes_per_symbol": 1.8881,
+        "bytes_per_symbol": 1.883,
         "source": "decode.cu",
-        "sha256_prefix": "b3b9f66f12b7c751"
+        "sha256_prefix": "10586da4d35c4248"
     },
     "encode_write_kernel": {
         "bytes_per_symbol": 2.0516,
         "source": "encode.cu",
-        "sha256_prefix": "bfd8deb88df791ab"
+        "sha256_prefix": "0c7c688082f50231"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0056,
@@ -136,12 +136,12 @@ MEASURED_TRAFFIC = {
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0001,
         "source": "build_tables.cu",
-        "sha256_prefix": "3365a0a098eabe33"
+        "sha256_prefix": "389cd91c45065dbd"
     },
     "encode_compact_kernel": {
-        "bytes_per_symbol": 1.782,
+        "bytes_per_symbol": 1.7818,
         "source": "encode.cu",
-        "sha256_prefix": "bfd8deb88df791ab"
+        "sha256_prefix": "0c7c688082f50231"
     }
 }
 

@@ -183,13 +183,18 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
     // (together ~257 candidate starts whatever g), and its threads take every 4th candidate of the
     // concatenated lists. Each thread scans its candidates in ascending j with a strict <, and the
     // group reduction prefers the smaller value, then the smaller j: the smallest j wins ties.
+    // Only end points i <= 256 - (K - k) can lie on a split into K non-empty ranges (the K - k ranges
+    // still to come need a symbol each), and every cell that does reads only such cells of the layer
+    // before; the cells above that band are never read, so they are not computed (at K = 256 the
+    // band is the single split into identity ranges).
     const int r4 = tid & 3;
     const int ia = 256 - (tid >> 2), ib = (tid >> 2) + 1;
     for (int k = 1; k <= K; ++k) {
       const long long* prev = S.drow[(k - 1) & 1];
       long long* cur = S.drow[k & 1];
-      const int na = (ia >= k) ? ((k == 1) ? 1 : ia - k + 1) : 0;  // j = k-1 .. (k == 1 ? 0 : i-1)
-      const int nb = (ib >= k) ? ((k == 1) ? 1 : ib - k + 1) : 0;
+      const int imax = 256 - (K - k);
+      const int na = (ia >= k && ia <= imax) ? ((k == 1) ? 1 : ia - k + 1) : 0;  // j = k-1 .. (k == 1 ? 0 : i-1)
+      const int nb = (ib >= k && ib <= imax) ? ((k == 1) ? 1 : ib - k + 1) : 0;
       long long best_a = LLONG_MAX, best_b = LLONG_MAX;
       int bj_a = 0x7fffffff, bj_b = 0x7fffffff;
       const uint32_t pa = S.pre[ia], pb = S.pre[ib];

@@ -171,10 +171,11 @@ __host__ __device__ inline SmemLayout smem_layout(uint32_t R, uint32_t K) {
 // Build decode tables (SHN1 format §5) for segments seg0 .. seg0+nt-1. replicated: nt == 1, entry of
 // slot i, replica c at byte (i*16 + c)*8; plain: table t at t*L*8, entry i at +i*8. All threads of
 // the block take part; the caller synchronises before (readers of the old tables are done).
-__device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, const SmemLayout& lay, uint32_t seg0,
+__device__ bool build_decode_tables(const uint8_t* recs, const DecHeader& h, const SmemLayout& lay, uint32_t seg0,
                                     uint32_t nt, bool replicated, unsigned char* dsm, uint32_t dsm_saddr) {
   const uint32_t K = h.K, R = h.R, L = 1u << R;
   const uint32_t tid = threadIdx.x;
+  bool wide = false;  // a range of these tables whose offset field does not fit beside R state bits in 16
   for (uint32_t e = tid; e < nt * K; e += blockDim.x) {
     const uint32_t t = e / K, k = e - t * K;
     const uint8_t* rec = recs + (uint64_t)h.tb * (seg0 + t);
@@ -183,10 +184,12 @@ __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, con
     uint32_t* wb = reinterpret_cast<uint32_t*>(sg + 2 * (K + 1) + 2 * K + ((2 * (K + 1) + 2 * K) & 2));
     const uint32_t lo = rec[2 * K + k];
     const uint32_t hi = (k + 1 < K) ? rec[2 * K + k + 1] : 256u;
+    const uint32_t w = width_bits(hi - lo);
     f[k] = (uint16_t)((uint32_t)rec[2 * k] | ((uint32_t)rec[2 * k + 1] << 8));
-    wb[k] = width_bits(hi - lo) | (((lo ^ 0x80u) & 0xFFu) << 8);
+    wb[k] = w | (((lo ^ 0x80u) & 0xFFu) << 8);
+    wide = wide || R + w > 16;
   }
-  __syncthreads();
+  const bool narrow = !__syncthreads_or(wide);
   for (uint32_t t = tid; t < nt; t += blockDim.x) {
     unsigned char* sg = dsm + lay.stage_off + t * lay.stage_per_table;
     uint16_t* cumul = reinterpret_cast<uint16_t*>(sg);
@@ -234,6 +237,7 @@ __device__ void build_decode_tables(const uint8_t* recs, const DecHeader& h, con
     }
   }
   __syncthreads();
+  return narrow;
 }
 
 // ---- per-thread chunk decoder -----------------------------------------------------------------
@@ -368,8 +372,8 @@ struct Fetcher {
       cp_async16(c.ring_saddr + (((uint32_t)lo * 16u) & (kRingBytes - 1)), c.comp + (uint64_t)(uint32_t)lo * 16u);
     }
   }
-  // Per 16-symbol piece at most N quads leave the ring (2 for fields of <= 16 bits, L <= 256; 3 for
-  // fields of <= 20 bits), so topping it up with at most N fetches keeps it full: no loop, N
+  // Per 16-symbol piece at most N quads leave the ring (2 for fields of <= 16 bits; 3 for fields of
+  // <= 20 bits), so topping it up with at most N fetches keeps it full: no loop, N
   // predicated copies.
   template <int N>
   __device__ __forceinline__ void top_up(const ChunkCtx& c, int32_t limit) {
@@ -384,8 +388,10 @@ struct Fetcher {
   }
 };
 
-// One chunk. SH = log2 of the table row stride in bytes. PAIRS (fields <= 16 bits, L <= 256): two
-// symbols per window position; otherwise one (fields <= 20 bits).
+// One chunk. SH = log2 of the table row stride in bytes. PAIRS (every symbol's state bits plus offset
+// bits fit in 16, i.e. R + widest offset <= 16: always for L <= 256, and for larger tables with
+// narrow ranges such as plain tANS): two symbols per window position; otherwise one (fields <= 20
+// bits).
 template <int S, int SH, bool PAIRS, class Sink>
 __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink& sk) {
   const uint32_t mask = kRingBytes - 1;
@@ -542,7 +548,8 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
     return;
   }
   const uint64_t n_tiles = (h.total_chunks + kDecThreads - 1) / kDecThreads;
-  int64_t cur_seg = -1;  // segment whose replicated table is in shared memory
+  uint32_t cur_seg = 0xFFFFFFFFu;  // segment whose replicated table is in shared memory (none: ~0 > n_segs - 1)
+  bool cur_pairs = false;  // whether its fields fit two to a 32-bit window read
   const uint64_t gmax = h.total_symbols > 0 ? (h.total_symbols - 1) >> o.gshift : 0;
   if (BF16 && h.total_symbols > 0 && gmax >= o.n_scales) {
     if (blockIdx.x == 0 && tid == 0) report(st, SHN_ERR_CAPACITY, 0);
@@ -603,35 +610,34 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
       }
     }
     if (sa == sb) {
-      if (cur_seg != (int64_t)sa) {
+      if (cur_seg != sa) {
         __syncthreads();
-        build_decode_tables(recs, h, lay, sa, 1, true, dsm, dsm_saddr);
+        cur_pairs = build_decode_tables(recs, h, lay, sa, 1, true, dsm, dsm_saddr);
         cur_seg = sa;
       }
       if (valid) {
         c.tbase = dsm_saddr + (lane & (dec_replicas(h.R) - 1)) * 8;
+        auto run_sh = [&](auto sh) { return cur_pairs ? run(c, sh, std::true_type()) : run(c, sh, std::false_type()); };
         bool ok;
-        using F = std::false_type;
-        using T = std::true_type;
         switch (h.R) {  // row stride: 16 copies x 8 bytes up to L = 256, then 8, 4, 2, 1 copies
-          case 9: ok = run(c, std::integral_constant<int, 6>(), F()); break;
-          case 10: ok = run(c, std::integral_constant<int, 5>(), F()); break;
-          case 11: ok = run(c, std::integral_constant<int, 4>(), F()); break;
-          case 12: ok = run(c, std::integral_constant<int, 3>(), F()); break;
-          default: ok = run(c, std::integral_constant<int, 7>(), T()); break;
+          case 9: ok = run_sh(std::integral_constant<int, 6>()); break;
+          case 10: ok = run_sh(std::integral_constant<int, 5>()); break;
+          case 11: ok = run_sh(std::integral_constant<int, 4>()); break;
+          case 12: ok = run_sh(std::integral_constant<int, 3>()); break;
+          default: ok = run(c, std::integral_constant<int, 7>(), std::true_type()); break;
         }
         if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
       }
     } else {
-      cur_seg = -1;
+      cur_seg = 0xFFFFFFFFu;
       for (uint32_t s0 = sa; s0 <= sb; s0 += lay.max_plain_tables) {
         const uint32_t nt = min(lay.max_plain_tables, sb - s0 + 1);
         __syncthreads();
-        build_decode_tables(recs, h, lay, s0, nt, false, dsm, dsm_saddr);
+        const bool pairs = build_decode_tables(recs, h, lay, s0, nt, false, dsm, dsm_saddr);
         if (valid && seg >= s0 && seg < s0 + nt) {
           c.tbase = dsm_saddr + (seg - s0) * L * 8;
-          const bool ok = h.R <= 8 ? run(c, std::integral_constant<int, 3>(), std::true_type())
-                                   : run(c, std::integral_constant<int, 3>(), std::false_type());
+          const bool ok = pairs ? run(c, std::integral_constant<int, 3>(), std::true_type())
+                                : run(c, std::integral_constant<int, 3>(), std::false_type());
           if (!ok) report(st, SHN_ERR_CORRUPT, (uint32_t)g);
         }
       }

@@ -87,8 +87,10 @@ struct Coder {
   }
 };
 
+// Returns whether every offset field this thread copied fits beside R state bits in 16 bits (the
+// block-wide AND of it decides whether two symbols' fields can share one 32-bit append).
 template <bool PLAIN>
-__device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table* t, uint32_t R, Coder<PLAIN>& cd) {
+__device__ __forceinline__ bool load_coder(unsigned char* smem, const shn_table* t, uint32_t R, Coder<PLAIN>& cd) {
   const uint32_t L = 1u << R;
   const uint32_t copies = PLAIN ? 1u : enc_copies(R);
   const uint32_t sym_copies = PLAIN ? 1u : kSymCopies;
@@ -96,7 +98,12 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   const uint16_t* enc = table_enc(t);
   uint2* s2 = reinterpret_cast<uint2*>(smem);
   unsigned char* e2 = smem + 256 * sym_copies * 8;
-  for (uint32_t i = threadIdx.x; i < 256 * sym_copies; i += blockDim.x) s2[i] = sym[i / sym_copies];
+  bool narrow = true;
+  for (uint32_t i = threadIdx.x; i < 256 * sym_copies; i += blockDim.x) {
+    const uint2 e = sym[i / sym_copies];
+    s2[i] = e;
+    narrow = narrow && R + ((e.y >> 8) & 0x7Fu) <= 16;  // bit 15 marks an absent byte, not width
+  }
   for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x)
     *reinterpret_cast<uint16_t*>(e2 + i * kEncSlot) = enc[i / copies];
   const uint32_t lane = threadIdx.x & 31;
@@ -105,6 +112,7 @@ __device__ __forceinline__ void load_coder(unsigned char* smem, const shn_table*
   // entry e of copy c is at e2 + (e * copies + c) * kEncSlot
   cd.enc = smem_addr(e2) + (lane & (copies - 1)) * kEncSlot - 4096u * cd.enc_row;
   cd.L = L;
+  return narrow;
 }
 
 // Run one chunk backwards (SHN1 format §6-§7), calling sink(field, width) for every field. seg points
@@ -148,7 +156,7 @@ __device__ __forceinline__ void code_chunk(const CoderT& cd, const uint8_t* seg,
   };
   auto code_piece = [&](const uint4 cur) {
     const uint32_t wv[4] = {cur.x, cur.y, cur.z, cur.w};
-    if (PAIRS) {  // symbols r and r-1: their fields (<= 16 bits each, L <= 256) as one append
+    if (PAIRS) {  // symbols r and r-1: their fields (<= 16 bits each) as one append
 #pragma unroll
       for (int r = 15; r >= 1; r -= 2) {
         const uint32_t b1 = __byte_perm(wv[r >> 2], 0u, 0x4440u + (uint32_t)(r & 3));
@@ -246,8 +254,7 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
   Coder<SMALL> cd;
-  load_coder(esm, t, lay.R, cd);
-  __syncthreads();
+  const bool narrow = __syncthreads_and(load_coder(esm, t, lay.R, cd));
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * NT + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
@@ -257,7 +264,8 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
   BitCounter bc;
-  code_chunk<S, PAIRS, true>(cd, in + b.offset[seg], geo, st, flags, bc);
+  if (PAIRS || narrow) code_chunk<S, true, true>(cd, in + b.offset[seg], geo, st, flags, bc);
+  else code_chunk<S, false, true>(cd, in + b.offset[seg], geo, st, flags, bc);
   const uint64_t total = (uint64_t)bc.bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
   if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
@@ -277,8 +285,7 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
   Coder<SMALL> cd;
-  load_coder(esm, t, lay.R, cd);
-  __syncthreads();
+  const bool narrow = __syncthreads_and(load_coder(esm, t, lay.R, cd));
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * NT + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
@@ -301,7 +308,8 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
 #pragma unroll
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
-  code_chunk<S, PAIRS, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
+  if (PAIRS || narrow) code_chunk<S, true, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
+  else code_chunk<S, false, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
 #pragma unroll
   for (int q = 0; q < S; ++q) rw(st[q] - cd.L, lay.R);
   rw(1u, 1u);  // sentinel
@@ -560,7 +568,8 @@ static cudaError_t launch_write_t(const uint8_t* d_in, const EncBatch& b, const 
                  : launch_write_small_t<S, PAIRS, SLOTS, false>(d_in, b, d_tables, lay, w, d_out, s);
 }
 
-// Two fields fit one 32-bit append when they are <= 16 bits each, i.e. L <= 256.
+// Two fields fit one 32-bit append when they are <= 16 bits each: always for L <= 256 (PAIRS); for
+// larger tables each block decides from its table's widest offset field.
 template <int S>
 static cudaError_t sizes_dispatch(const uint8_t* d_in, const EncBatch& b, const shn_table* t, const EncodeLayout& lay,
                                   const EncodeWork& w, cudaStream_t s) {

@@ -114,14 +114,36 @@ def test_config2_plain_tans_l1024(orc):
 @pytest.mark.parametrize("K,R,S,C", [(256, 9, 4, 1024), (16, 10, 2, 4096), (200, 11, 8, 256), (256, 12, 1, 128),
                                      (3, 12, 16, 1024), (32, 9, 4, 65536)])
 def test_large_state_counts(orc, K, R, S, C):
-    """L = 512 ... 4096: fields up to R + 8 bits, one symbol per window position, fewer table copies;
-    ragged segments so tiles straddle segments (plain per-segment tables)."""
+    """L = 512 ... 4096: fields up to R + 8 bits, fewer table copies; two symbols per window position
+    where R plus the widest offset fits 16 bits (K = 256, 200, 32 here), one otherwise (K = 3); ragged
+    segments so tiles straddle segments (plain per-segment tables)."""
     rng = np.random.default_rng(K + 7 * R)
     n = 200_003
     x = inputs.laplace_int8(n, float(rng.choice([3.0, 20.0, 97.0])), seed=K * R).numpy()
     cuts = sorted(set([0, n] + rng.integers(0, n, 4).tolist()))
     segs = [(a, b - a) for a, b in zip(cuts[:-1], cuts[1:])]
     check_parity(orc, x, segs, shn.CodecParams(K, R, C, S))
+
+
+@pytest.mark.parametrize("R", [9, 10, 11, 12])
+def test_large_tables_mixed_field_widths(orc, R):
+    """One L > 256 stream whose segment tables differ in their widest offset field: a near-uniform
+    segment (ranges of ~16 symbols) beside a peaked one (its empty tails become ranges of > 64
+    symbols), and small segments. With 128-symbol chunks the two large segments fill whole decoder
+    tiles (one replicated table) and the small ones share tiles (several tables). Encoder blocks
+    choose paired or single field appends per table, decoder tiles per set of tables; the stream
+    must not depend on either choice."""
+    sizes_b = [(150_000, 97.17), (150_000, 0.7), (3_000, 97.17), (2_500, 0.7), (40_000, 20.0), (777, 0.7)]
+    x = np.concatenate([inputs.laplace_int8(n, b, seed=10 * R + i).numpy() for i, (n, b) in enumerate(sizes_b)])
+    cuts = np.cumsum([0] + [n for n, _ in sizes_b])
+    segs = [(int(a), int(b - a)) for a, b in zip(cuts[:-1], cuts[1:])]
+    g, _ = check_parity(orc, x, segs, shn.CodecParams(16, R, 128, 4))
+    widest = []
+    for t in g["tables"]:
+        lo = list(t["lo"]) + [256]
+        widest.append(max(int(np.ceil(np.log2(b - a))) if b - a > 1 else 0 for a, b in zip(lo[:-1], lo[1:])))
+    if R in (10, 11):  # both kinds of table are present
+        assert min(widest) + R <= 16 < max(widest) + R, widest
 
 
 def test_config4_activation_batch_full(orc):
