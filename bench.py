@@ -729,6 +729,19 @@ def main():
             stages[k] = {"ms": ms, "gbs_int8": n / (ms * 1e-3) / 1e9 if ms > 0 else None}
         alg = {"histogram": n, "build": 0, "encode": n + nbytes, "decode": n + nbytes}
         dom = max(("encode", "decode", "histogram"), key=lambda k: stages[k]["ms"])
+        if offl is not None:
+            # Shannonic §6, when compression pays: sender encodes, the link carries CSR of the bytes,
+            # the receiver decodes, one after the other; with every rate INT8-side that is
+            # CSR < 1 - R_link (1/R_enc + 1/R_dec). R_enc covers histogram + tables + encode.
+            ms_enc = stages["histogram"]["ms"] + stages["build"]["ms"] + stages["encode"]["ms"]
+            ms_dec = stages["decode"]["ms"]
+            csr = offl["compressed_bytes"] / n
+            cond = {"csr": csr, "r_enc_gbs": n / ms_enc / 1e6, "r_dec_gbs": n / ms_dec / 1e6}
+            for d in ("d2h", "h2d"):
+                r_link = n / offl[f"raw_{d}_ms"] / 1e6
+                csr_max = 1.0 - r_link * (1.0 / cond["r_enc_gbs"] + 1.0 / cond["r_dec_gbs"])
+                cond[d] = {"r_link_gbs": r_link, "csr_max": csr_max, "pays": bool(csr < csr_max)}
+            offl["latency_condition"] = cond
 
         kernels_of = {"decode": ["decode_kernel"], "encode": ["encode_write_kernel", "encode_compact_kernel"],
                       "histogram": ["histogram_kernel"]}
