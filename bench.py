@@ -136,7 +136,7 @@ MEASURED_TRAFFIC = {
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0001,
         "source": "build_tables.cu",
-        "sha256_prefix": "389cd91c45065dbd"
+        "sha256_prefix": "bd749e6febc66f81"
     },
     "encode_compact_kernel": {
         "bytes_per_symbol": 1.7818,

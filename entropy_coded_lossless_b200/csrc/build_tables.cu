@@ -71,32 +71,65 @@ __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L
 #pragma unroll
     for (int r = 0; r < kPer; ++r) f[r] = (tid == 0 && r == 0) ? L : 0u;
   } else {
-    // K <= L is checked on the host, so nonzero <= L
-    for (uint32_t step = 0; step < L - (uint32_t)nonzero; ++step) {
-      unsigned long long bg = 0;
-      int bk = 0x7fffffff;
+    // K <= L is checked on the host, so nonzero <= L. G[r] caches the gain of the next state of
+    // range tid + 32 r (0 for an empty range; every other gain is > 0, as LG is strictly increasing).
+    // Only the winning range's gain changes in a step, so one gain is recomputed per step.
+    unsigned long long G[kPer];
+#pragma unroll
+    for (int r = 0; r < kPer; ++r)
+      G[r] = N[r] > 0 ? N[r] * (unsigned long long)(S.lgf[f[r] + 1] - S.lgf[f[r]]) : 0ull;
+    unsigned long long bg;
+    int bk;
+    auto rescan = [&]() {  // largest cached gain of this lane, ties to the smallest k (tournament, left wins ties)
+      unsigned long long gv[kPer];
+      int kv[kPer];
 #pragma unroll
       for (int r = 0; r < kPer; ++r) {
-        const int k = tid + 32 * r;
-        if (N[r] > 0) {
-          const unsigned long long g = N[r] * (unsigned long long)(S.lgf[f[r] + 1] - S.lgf[f[r]]);
-          if (bk == 0x7fffffff || g > bg || (g == bg && k < bk)) {
-            bg = g;
-            bk = k;
-          }
-        }
+        gv[r] = G[r];
+        kv[r] = tid + 32 * r;
       }
+#pragma unroll
+      for (int w = 1; w < kPer; w <<= 1)
+#pragma unroll
+        for (int r = 0; r + w < kPer; r += 2 * w)
+          if (gv[r + w] > gv[r]) {
+            gv[r] = gv[r + w];
+            kv[r] = kv[r + w];
+          }
+      bg = gv[0];
+      bk = gv[0] > 0 ? kv[0] : 0x7fffffff;
+    };
+    rescan();
+    for (uint32_t step = 0; step < L - (uint32_t)nonzero; ++step) {
       // warp argmax of (gain, then smallest k) with three reductions: the high word of the gain,
       // the low word among lanes at that high word, the smallest k among lanes at the maximum.
-      // Every valid gain is > 0 (N_k > 0 and LG strictly increasing), lanes without one hold 0.
       const uint32_t ghi = (uint32_t)(bg >> 32), glo = (uint32_t)bg;
       const uint32_t m1 = __reduce_max_sync(0xffffffffu, ghi);
       const uint32_t m2 = __reduce_max_sync(0xffffffffu, ghi == m1 ? glo : 0u);
-      bk = (int)__reduce_min_sync(0xffffffffu, (ghi == m1 && glo == m2 && bk != 0x7fffffff) ? (uint32_t)bk
-                                                                                                 : 0xffffffffu);
+      const int win = (int)__reduce_min_sync(0xffffffffu, (ghi == m1 && glo == m2 && bk != 0x7fffffff) ? (uint32_t)bk
+                                                                                                        : 0xffffffffu);
+      // The winning range's lane gives it one more state and caches its next gain. Every lane runs
+      // the same instructions (no divergence); on the others the writes are predicated off and the
+      // rescan finds the best it already had.
+      const bool mine = (win & 31) == tid;
+      const int rw = win >> 5;
+      uint32_t fw = f[0];
+      unsigned long long nw = N[0];
+#pragma unroll
+      for (int r = 1; r < kPer; ++r)
+        if (r == rw) {
+          fw = f[r];
+          nw = N[r];
+        }
+      fw += 1;  // on the winner, fw == L only after the last step (lgf has L + 1 entries)
+      const unsigned long long gw = fw < L ? nw * (unsigned long long)(S.lgf[fw + 1] - S.lgf[fw]) : 0ull;
 #pragma unroll
       for (int r = 0; r < kPer; ++r)
-        if (tid + 32 * r == bk) f[r] += 1;
+        if (mine && r == rw) {
+          f[r] = fw;
+          G[r] = gw;
+        }
+      rescan();
     }
   }
 #pragma unroll

@@ -43,7 +43,7 @@ typedef enum shn_status {
   SHN_ERR_CORRUPT = 3,     /* the compressed stream fails a structural or end-of-chunk check */
   SHN_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
   SHN_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reserved; current kernels never wait) */
-  SHN_ERR_UNSUPPORTED = 6, /* valid parameters this build's kernels do not implement */
+  SHN_ERR_UNSUPPORTED = 6, /* valid parameters that the library's kernels do not implement */
   SHN_ERR_WORKSPACE = 7    /* the workspace is smaller than the *_workspace_bytes query returned */
 } shn_status;
 
