@@ -99,6 +99,25 @@ def workload(name, device, seed_offset=0, n_segments=0, entropy=5.3):
     return x, segs, dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4), desc
 
 
+def kernel_launches_per_step(segs, p_dict) -> int:
+    """Kernels one step launches through the four calls, following the library's batching: a
+    histogram launch per 512 segments; the table build (plus the LG-table fill from 256 tables on);
+    per encoder batch (at most 512 consecutive segments of one kind, where segments of at most 64
+    chunks, empty ones included, are the small kind) a slot-coding launch and a header launch; the
+    three-launch scan and the slot compaction once; the decoder's check and decode launches."""
+    n = len(segs)
+    if n == 0:
+        return 0
+    launches = -(-n // 512) + 1 + (1 if n >= 256 else 0) + 3 + 1 + 2
+    batches, count, kind = 0, 0, None
+    for _, length in segs:
+        small = -(-length // p_dict["chunk_symbols"]) <= 64
+        if batches == 0 or count == 512 or small != kind:
+            batches, count, kind = batches + 1, 0, small
+        count += 1
+    return launches + 2 * batches
+
+
 def max_over_ranks(value: float, device) -> float:
     """Max of a per-rank float over the process group (identity without one)."""
     if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
@@ -754,7 +773,7 @@ def main():
                     "alg_bytes_per_launch": alg[k], "peak_kind": peak_kind,
                     "timing": "CUDA events around the C-ABI call on the launching stream, mean over the timed steps"}
 
-        launches_per_step = 1 + 1 + 1 + 3 + 1 + 1 + 2  # hist, build, sizes, scan x3, header, write, check+decode
+        launches_per_step = kernel_launches_per_step(segs, p_dict)
         line = {
             "metric": METRIC,
             "value": whole_job_gbs(n, world, ms_step),
