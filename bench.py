@@ -118,6 +118,22 @@ def kernel_launches_per_step(segs, p_dict) -> int:
     return launches + 2 * batches
 
 
+# seed of each workload's generator (rank r of a multi-GPU run adds r)
+WORKLOAD_SEED = {"kv": 2, "weight": 1, "int4": 6, "activations": 3, "sweep": 4}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def max_over_ranks(value: float, device) -> float:
     """Max of a per-rank float over the process group (identity without one)."""
     if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
@@ -322,7 +338,7 @@ def cpu_baseline(x_dev, segs, p, budget_s, full_n):
     dt = time.perf_counter() - t
     assert rc == 0 and np.array_equal(y, xs.view(np.uint8))
     nbytes = xs.size
-    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{k} of {len(segs)} segments ({nbytes} bytes): histogram+DP+tables+encode+decode, "
                       f"{dt:.1f} s on {cores} host threads"}
 
@@ -460,8 +476,9 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
             "config": {"workload": desc, "K": p["K"], "L": 1 << p["log2L"], "chunk_symbols": p["chunk_symbols"],
-                       "states_per_chunk": p["states_per_chunk"], "sample_segments": k},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                       "states_per_chunk": p["states_per_chunk"], "sample_segments": k,
+                       "seed": WORKLOAD_SEED.get(args.workload)},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"{k} of {len(segs)} segments per step ({xs.size} bytes)"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -789,6 +806,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": desc, "K": p.K, "L": 1 << p.log2L, "chunk_symbols": p.chunk_symbols,
                        "states_per_chunk": p.states_per_chunk, "bytes_per_gpu": n,
+                       "seed": None if WORKLOAD_SEED.get(args.workload) is None else WORKLOAD_SEED[args.workload] + rank,
                        "l2": "inputs larger than L2 (input, stream and output each > 126 MB per step)"
                        if flush is None else "L2 flushed (256 MiB write) before every step; step time = sum of stage events",
                        "parallelism": f"replicas x{world} (independent segments per rank)"},
