@@ -401,7 +401,9 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
   fe.bottom = (int32_t)(c.cb >> 4);
   fe.lo = q_top + 1;
   fe.fill_to(c, q_top - (int32_t)kRingQuads + 1);
-  const int32_t cb_words = (int32_t)(c.cb >> 2);  // chunk start in stream words
+  // quad of the window's low word: bottom + (chunk start word within its quad + window word) / 4,
+  // kept in 32 bits for streams up to 32 GiB (the chunk's word offset alone would not be)
+  const int32_t cb_wq = (int32_t)((c.cb >> 2) & 3u);
   cp_async_commit();
   cp_async_wait<0>();
   // ring address of chunk word k (k may be negative: a stale word, never used validly)
@@ -432,7 +434,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
   const uint32_t full = c.pieces - (c.last_len < 16 ? 1u : 0u);
   sk.start(c);
   for (uint32_t k = 0; k < full; ++k) {
-    fe.top_up<PAIRS ? 2 : 3>(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    fe.top_up<PAIRS ? 2 : 3>(c, fe.bottom + ((cb_wq + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<1>();
     sk.begin_piece();
@@ -479,7 +481,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
     sk.end_piece();
   }
   if (full < c.pieces) {  // the group's short last piece
-    fe.fill_to(c, ((cb_words + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
+    fe.fill_to(c, fe.bottom + ((cb_wq + (thr >> 5)) >> 2) - (int32_t)kRingQuads + 1);
     cp_async_commit();
     cp_async_wait<0>();
     for (uint32_t i = 0; i < c.last_len; ++i) {

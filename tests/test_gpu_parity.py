@@ -265,6 +265,26 @@ def test_config5_full_gib(orc):
     _full_size(orc, x, [(0, x.numel())], shn.CodecParams(16, 7, 4096, 4), table_check_segs=[0])
 
 
+def test_segments_beyond_2gib(orc):
+    """3 GiB in two segments, the second starting past 2^31 bytes and the stream running past 2^32
+    bits, with a ragged tail: 64-bit offsets throughout (an int32 overflow anywhere in the path
+    would show here as a wrong histogram, a failed round trip or a sampled chunk that differs)."""
+    n1, n2 = (1 << 31) + 48, (1 << 30) + 12_345
+    x = inputs.laplace_int8(n1 + n2, inputs.LAPLACE_B_FOR_ENTROPY[5.3], seed=12, device=DEV)
+    nbytes = _full_size(orc, x, [(0, n1), (n1, n2)], shn.CodecParams(16, 7, 4096, 4), table_check_segs=[0, 1])
+    assert nbytes > (1 << 31)
+
+def test_stream_beyond_8gib(orc):
+    """8.4 GiB of near-uniform bytes (H = 7.9 bits) in three segments: a stream of ~8.3 GiB, past
+    where byte offsets divided by 4 leave 32-bit signed range. The encoder accepts any input whose
+    worst-case bound (15 bits per value at L = 128) stays within 16 GiB, i.e. up to ~8.5 GiB, and
+    near-incompressible input gives a stream of about its own size."""
+    n = int(2.8 * (1 << 30)) & ~15
+    segs = [(0, n), (n, n), (2 * n, n + 12_345)]
+    x = inputs.laplace_int8(3 * n + 12_345, inputs.LAPLACE_B_FOR_ENTROPY[7.9], seed=13, device=DEV)
+    nbytes = _full_size(orc, x, segs, shn.CodecParams(16, 7, 4096, 4), table_check_segs=[2])
+    assert nbytes > (8 << 30)
+
 # ---- errors reported on the device ------------------------------------------------------------
 
 
