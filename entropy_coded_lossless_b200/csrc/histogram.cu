@@ -11,8 +11,10 @@
 namespace shn {
 
 constexpr int kHistThreadsPerBlock = 512;
-constexpr uint32_t kHistVecPerThread = 16;  // 16 B each
-constexpr uint32_t kHistBytesPerBlock = kHistThreadsPerBlock * 16 * kHistVecPerThread;  // 128 KiB
+// 16-byte vectors per thread: 512 KiB per block, so that zeroing and folding the block's 8192
+// counters is small beside its loads (measured: 92 % of the copy bandwidth, against 85 % at 128 KiB)
+constexpr uint32_t kHistVecPerThread = 64;
+constexpr uint32_t kHistBytesPerBlock = kHistThreadsPerBlock * 16 * kHistVecPerThread;
 
 __device__ __forceinline__ void count_word(uint32_t* col, uint32_t w) {
   atomicAdd(col + ((w & 0xFFu) << 5), 1u);
