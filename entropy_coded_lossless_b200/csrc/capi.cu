@@ -117,13 +117,16 @@ int shn_histogram(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_seg
   for (uint32_t s0 = 0; s0 < n_segs; s0 += kSegBatch) {
     memset(&b, 0, sizeof(b));
     b.n = (n_segs - s0 < (uint32_t)kSegBatch) ? n_segs - s0 : (uint32_t)kSegBatch;
+    uint64_t bytes = 0;
+    for (uint32_t i = 0; i < b.n; ++i) bytes += h_segs[s0 + i].length;
+    b.bytes_per_block = histogram_bytes_per_block(bytes, sm_count());
     uint64_t blocks = 0;
     for (uint32_t i = 0; i < b.n; ++i) {
       b.offset[i] = h_segs[s0 + i].offset;
       b.length[i] = (uint32_t)h_segs[s0 + i].length;
       b.block_start[i] = (uint32_t)blocks;
       b.hist_index[i] = s0 + i;
-      blocks += histogram_blocks_for(h_segs[s0 + i].length);
+      blocks += histogram_blocks_for(h_segs[s0 + i].length, b.bytes_per_block);
     }
     if (blocks >= (1ull << 31)) return SHN_ERR_INVALID_ARG;
     b.total_blocks = (uint32_t)blocks;

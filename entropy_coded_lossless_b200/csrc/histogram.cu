@@ -11,10 +11,13 @@
 namespace shn {
 
 constexpr int kHistThreadsPerBlock = 512;
-// 16-byte vectors per thread: 512 KiB per block, so that zeroing and folding the block's 8192
-// counters is small beside its loads (measured: 92 % of the copy bandwidth, against 85 % at 128 KiB)
-constexpr uint32_t kHistVecPerThread = 64;
-constexpr uint32_t kHistBytesPerBlock = kHistThreadsPerBlock * 16 * kHistVecPerThread;
+// Bytes per block: as many as keep at least kHistMinBlocksPerSm blocks per SM busy, up to 512 KiB,
+// so that zeroing and folding the block's 8192 counters is small beside its loads (measured on the
+// 2 GiB KV cache: 92 % of the copy bandwidth at 512 KiB, 85 % at 128 KiB); small tensors get
+// blocks down to 32 KiB instead of leaving most SMs idle.
+constexpr uint32_t kHistMaxBytesPerBlock = 512u << 10;
+constexpr uint32_t kHistMinBytesPerBlock = 32u << 10;
+constexpr uint64_t kHistMinBlocksPerSm = 4;
 
 __device__ __forceinline__ void count_word(uint32_t* col, uint32_t w) {
   atomicAdd(col + ((w & 0xFFu) << 5), 1u);
@@ -38,8 +41,8 @@ __global__ void __launch_bounds__(kHistThreadsPerBlock) histogram_kernel(const u
   const uint32_t part = blockIdx.x - b.block_start[seg];
   const uint64_t seg_begin = b.offset[seg];
   const uint64_t seg_end = seg_begin + b.length[seg];
-  const uint64_t begin = seg_begin + (uint64_t)part * kHistBytesPerBlock;
-  const uint64_t end = min(seg_end, begin + kHistBytesPerBlock);
+  const uint64_t begin = seg_begin + (uint64_t)part * b.bytes_per_block;
+  const uint64_t end = min(seg_end, begin + b.bytes_per_block);
 
   for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) sh[i] = 0;
   __syncthreads();
@@ -93,6 +96,15 @@ cudaError_t launch_histogram(const uint8_t* d_in, const HistBatch& b, uint64_t* 
   return cudaGetLastError();
 }
 
-uint32_t histogram_blocks_for(uint64_t length) { return (uint32_t)((length + kHistBytesPerBlock - 1) / kHistBytesPerBlock); }
+uint32_t histogram_bytes_per_block(uint64_t batch_bytes, int sm_count) {
+  uint32_t bpb = kHistMaxBytesPerBlock;
+  const uint64_t want = kHistMinBlocksPerSm * (uint64_t)(sm_count > 0 ? sm_count : 1);
+  while (bpb > kHistMinBytesPerBlock && batch_bytes / bpb < want) bpb >>= 1;
+  return bpb;
+}
+
+uint32_t histogram_blocks_for(uint64_t length, uint32_t bytes_per_block) {
+  return (uint32_t)((length + bytes_per_block - 1) / bytes_per_block);
+}
 
 }  // namespace shn

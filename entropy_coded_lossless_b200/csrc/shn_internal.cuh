@@ -162,6 +162,7 @@ struct HistBatch {
   uint32_t length[kSegBatch];      // bytes
   uint32_t block_start[kSegBatch]; // first block of each segment
   uint32_t hist_index[kSegBatch];  // histogram row of each segment
+  uint32_t bytes_per_block;        // input bytes per block (histogram_bytes_per_block)
 };
 
 struct EncBatch {
@@ -179,7 +180,8 @@ struct EncBatch {
 // Launch wrappers (defined in the .cu files; return a cudaError_t).
 cudaError_t launch_histogram(const uint8_t* d_in, const HistBatch& b, uint64_t* d_hist, int threads,
                              cudaStream_t s);
-uint32_t histogram_blocks_for(uint64_t length);
+uint32_t histogram_bytes_per_block(uint64_t batch_bytes, int sm_count);
+uint32_t histogram_blocks_for(uint64_t length, uint32_t bytes_per_block);
 cudaError_t launch_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params& p,
                                 shn_table* d_tables, cudaStream_t s);
 
