@@ -159,9 +159,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "df7d582782b48517"
     },
     "encode_write_kernel": {
-        "bytes_per_symbol": 2.0515,
+        "bytes_per_symbol": 2.0535,
         "source": "encode.cu",
-        "sha256_prefix": "c80ee9d5885ed821"
+        "sha256_prefix": "7bd0eed599b12aac"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0031,
@@ -174,9 +174,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "bd749e6febc66f81"
     },
     "encode_compact_kernel": {
-        "bytes_per_symbol": 1.7821,
+        "bytes_per_symbol": 1.7811,
         "source": "encode.cu",
-        "sha256_prefix": "c80ee9d5885ed821"
+        "sha256_prefix": "7bd0eed599b12aac"
     }
 }
 
