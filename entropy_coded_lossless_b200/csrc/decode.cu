@@ -1,5 +1,5 @@
-// decode.cu — chunk-parallel Shannonic/tANS decoder (Shannonic §4.2: "from state X, decTable[X]
-// gives the symbol s and the bit count; read the offset o and restore x = base[s] + o").
+// decode.cu — chunk-parallel Shannonic/tANS decoder (Shannonic §4.2, decoding: the decode table
+// entry of the state gives the range s and its bit count, the offset o follows, x = base[s] + o).
 //
 // Work layout. A persistent grid of 256-thread blocks walks tiles of 256 consecutive chunks; each
 // thread decodes one chunk of C symbols with S interleaved states (SHN1 format §7), reading the chunk
@@ -12,17 +12,19 @@
 // fields above bit 7 are written as multiply-highs (y >> s == mulhi(y, 2^(32-s)), and a signed
 // mulhi by 2^8 yields the negated field width); the compiler chooses shift or integer-multiply
 // instructions for them (forcing the multiply pipe for all of them measured slower). When a tile lies
-// in one segment (the common case for large tensors) the table is stored 16 times interleaved
-// ([slot][replica], replica = lane & 15): an 8-byte load is served per half-warp, so the 16 lanes of
-// a half-warp always hit 16 different bank pairs whatever their states — no bank conflicts. Tiles
-// that straddle segments (many small tensors) use plain per-segment copies, built up to 16 at a
-// time. Tables are built in shared memory from the (f, lo) records of the stream.
+// in one segment (the common case for large tensors) the table is stored interleaved
+// ([slot][replica], replica = lane & (copies - 1)): 16 copies up to L = 512, where an 8-byte load
+// is served per half-warp and the 16 lanes of a half-warp always hit 16 different bank pairs
+// whatever their states (no bank conflicts); 8, 4, 2 copies at L = 1024 ... 4096 (a 64 KB table).
+// Tiles that straddle segments (many small tensors) use plain per-segment copies, built up to 16 at
+// a time. Tables are built in shared memory from the (f, lo) records of the stream.
 //
 // Bits. Each thread keeps a 64-bit window (two words) of its chunk in registers and refills it from
 // a private 128-byte ring in shared memory, which cp.async (16-byte, L2-only) copies fill ahead of
 // use. All shared-memory accesses of the per-symbol loop use 32-bit shared-window addresses. Two
-// symbols are extracted per window position when fields are <= 16 bits (L <= 256), one otherwise
-// (fields <= 20 bits, L <= 4096). Decoded values go to an output sink: the INT8 tensor (16-byte
+// symbols are extracted per window position when every field fits 16 bits (R plus the widest
+// offset of the tables in shared memory: always at L <= 256), one otherwise (fields <= 20 bits,
+// L <= 4096). Decoded values go to an output sink: the INT8 tensor (16-byte
 // stores of 16 values) or, fused with the consumer, bf16 values dequantised by a per-group scale.
 //
 // Robustness. Corrupt input never causes an out-of-bounds access: descriptors and the chunk index

@@ -1,5 +1,5 @@
-// histogram.cu — 256-bin histogram of INT8 segments (Shannonic §4.1: "compute the histogram h[x]
-// of the input tensor"; symbol u = byte ^ 0x80, SHN1 format §1).
+// histogram.cu — 256-bin histogram of INT8 segments, the first preprocessing step of Shannonic
+// §4.1 (counts of every value of the tensor); symbol u = byte ^ 0x80, SHN1 format §1.
 //
 // HBM-bound: every input byte is read once with 128-bit loads. Each block keeps a lane-private
 // histogram in shared memory laid out [byte value][lane], so a warp's 32 increments always land in

@@ -109,8 +109,8 @@ size_t shn_decode_workspace_bytes(const shn_params* p);
 /* --- the codec ---------------------------------------------------------------------------- */
 
 /*
- * 256-bin histogram of each segment (Shannonic §4.1: "compute the histogram h[x] of the input
- * tensor"). d_hist[s*256 + u] = number of bytes b in segment s with (b ^ 0x80) == u.
+ * 256-bin histogram of each segment (Shannonic §4.1, the preprocessing step that counts every
+ * value of the tensor). d_hist[s*256 + u] = number of bytes b in segment s with (b ^ 0x80) == u.
  *  d_in    device, the input bytes; any alignment.
  *  h_segs  host array of n_segs segments; every segment must lie inside d_in's allocation.
  *  d_hist  device, n_segs*256 uint64, 8-byte aligned; fully overwritten.
