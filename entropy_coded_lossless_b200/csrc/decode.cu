@@ -15,7 +15,10 @@
 // in one segment (the common case for large tensors) the table is stored interleaved
 // ([slot][replica], replica = lane & (copies - 1)): 16 copies up to L = 512, where an 8-byte load
 // is served per half-warp and the 16 lanes of a half-warp always hit 16 different bank pairs
-// whatever their states (no bank conflicts); 8, 4, 2 copies at L = 1024 ... 4096 (a 64 KB table).
+// whatever their states (table lookups never conflict); 8, 4, 2 copies at L = 1024 ... 4096 (a 64 KB
+// table). The bank conflicts ncu counts in this kernel (about a fifth of its shared wavefronts on the
+// KV cache) come from the window refills: lanes whose rings are at the same word offset meet on one
+// bank. They cost LSU cycles, not ALU ones, and the kernel is ALU-bound.
 // Tiles that straddle segments (many small tensors) use plain per-segment copies, built up to 16 at
 // a time. Tables are built in shared memory from the (f, lo) records of the stream.
 //
