@@ -1,0 +1,149 @@
+"""The CUDA kernels compute some steps in a different order or form than the oracle does. These CPU
+tests restate those forms in Python, from their description in the kernel sources, and check them
+against the oracle on random inputs, so that each reformulation is shown to give the oracle's
+result exactly (the GPU parity tests then check the kernels themselves):
+
+* the greedy state allocation with cached per-range gains and a per-lane tournament
+  (build_tables.cu, normalize_warp) against the oracle's sequential greedy;
+* the range DP restricted to the end points that can still lie on a split into K non-empty
+  ranges (build_tables.cu) against the oracle's full DP;
+* the decoder's ring-refill quad index, kept in 32 bits (decode.cu), against the plain formula.
+"""
+import numpy as np
+import pytest
+
+INF = 1 << 80
+
+
+def lg_table(orc, L):
+    return [orc.lg(f) for f in range(L + 2)]
+
+
+def tournament_greedy(N, R, lgf):
+    """Lane l holds ranges l + 32 r (r < kPer); every lane caches the gain of each of its ranges and
+    its best (largest gain, then smallest k, by a left-priority tournament); a step is a warp argmax
+    over the lanes' bests (largest gain, then smallest k); only the winner's gain is recomputed."""
+    K = len(N)
+    L = 1 << R
+    kper = 1 if K <= 32 else 2 if K <= 64 else 4 if K <= 128 else 8
+    n = [int(N[k]) if k < K else 0 for k in range(32 * kper)]
+    f = [1 if v > 0 else 0 for v in n]
+    if sum(n) == 0:
+        out = [0] * K
+        out[0] = L
+        return out
+
+    def gain(k):
+        return n[k] * (lgf[f[k] + 1] - lgf[f[k]]) if n[k] > 0 and f[k] < L else 0
+
+    G = [gain(k) for k in range(32 * kper)]
+
+    def lane_best(lane):
+        gv = [G[lane + 32 * r] for r in range(kper)]
+        kv = [lane + 32 * r for r in range(kper)]
+        w = 1
+        while w < kper:
+            for r in range(0, kper - w, 2 * w):
+                if gv[r + w] > gv[r]:
+                    gv[r], kv[r] = gv[r + w], kv[r + w]
+            w *= 2
+        return gv[0], (kv[0] if gv[0] > 0 else None)
+
+    best = [lane_best(lane) for lane in range(32)]
+    for _ in range(L - sum(f)):
+        top = max(g for g, _ in best)
+        win = min(k for g, k in best if g == top and k is not None)
+        f[win] += 1
+        G[win] = gain(win)
+        best[win & 31] = lane_best(win & 31)
+    return f[:K]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_tournament_greedy_matches_oracle(orc, seed):
+    rng = np.random.default_rng(seed)
+    K = int(rng.choice([1, 3, 16, 31, 33, 64, 100, 129, 200, 256]))
+    R = int(rng.integers(max(4, int(np.ceil(np.log2(K)))), 11))
+    top = min(1 << int(rng.choice([6, 20, 31])), (1 << 32) // (K + 1))  # the total stays below 2^32
+    pool = rng.integers(1, top, 4)  # few distinct counts: many ties
+    N = rng.choice(np.concatenate([[0, 0, 1], pool]), K).astype(np.uint64)
+    if int((N > 0).sum()) > (1 << R):
+        N[(1 << R):] = 0
+    expect = orc.normalize(N, R)
+    got = tournament_greedy(N, R, lg_table(orc, 1 << R))
+    assert list(expect) == got
+
+
+def banded_dp(orc, h, K):
+    """The kernel's layer order: D[i][k] = min over j in [k-1, i-1] of D[j][k-1] + Cost(j, i), ties to
+    the smallest j, computed only for k <= i <= 256 - (K - k); backtrack from D[256][K]."""
+    A = len(h)
+    pre = np.concatenate([[0], np.cumsum(h.astype(np.int64))])
+    lgs = {}
+
+    def cost(j, i):
+        c = int(pre[i] - pre[j])
+        if c == 0:
+            return 0
+        if c not in lgs:
+            lgs[c] = orc.lg(c)
+        width = i - j
+        w = 0 if width <= 1 else int(width - 1).bit_length()
+        return c * ((w << 24) - lgs[c])
+
+    prev = [0] + [INF] * A
+    arg = []
+    for k in range(1, K + 1):
+        cur = [INF] * (A + 1)
+        a_k = {}
+        for i in range(k, A - (K - k) + 1):
+            best, bj = INF, None
+            for j in range(k - 1, i):
+                if prev[j] >= INF:
+                    continue
+                v = prev[j] + cost(j, i)
+                if v < best:
+                    best, bj = v, j
+            cur[i], a_k[i] = best, bj
+        arg.append(a_k)
+        prev = cur
+    lo, i = [0] * K, A
+    for k in range(K, 0, -1):
+        j = arg[k - 1][i]
+        lo[k - 1] = j
+        i = j
+    return lo, prev[A]
+
+
+@pytest.mark.parametrize("seed,K", [(0, 1), (1, 2), (2, 5), (3, 8), (4, 12), (5, 15), (6, 16)])
+def test_banded_dp_matches_oracle_small_alphabet(orc, seed, K):
+    # a 16-symbol alphabet keeps the pure-Python DP fast while every band edge is exercised
+    rng = np.random.default_rng(100 + seed)
+    h = rng.choice([0, 0, 1, 7, 1000, 123456], 16).astype(np.uint64)
+    lo_o, cost_o = orc.partition(h, K)
+    lo, cost = banded_dp(orc, h, K)
+    assert cost == cost_o and lo == [int(v) for v in lo_o]
+
+
+def test_banded_dp_matches_oracle_full_alphabet(orc):
+    rng = np.random.default_rng(7)
+    v = np.clip(np.round(rng.laplace(0, 9, 20000)), -128, 127).astype(np.int64) + 128
+    h = np.bincount(v, minlength=256).astype(np.uint64)
+    for K in (250, 255, 256):  # narrow bands, where the restriction drops most cells
+        lo_o, cost_o = orc.partition(h, K)
+        lo, cost = banded_dp(orc, h, K)
+        assert cost == cost_o and lo == [int(x) for x in lo_o], K
+
+
+def test_refill_quad_index_in_32_bits():
+    """quad((cb / 4 + t)) = (cb / 4 + t) >> 2 equals (cb >> 4) + (((cb >> 2) & 3) + t) >> 2 for 4-byte
+    aligned chunk starts cb anywhere below 32 GiB and window words t, negative ones included (Python
+    >> floors like an arithmetic shift)."""
+    rng = np.random.default_rng(3)
+    cbs = [4 * int(x) for x in rng.integers(0, (32 << 30) // 4, 2000)] + [0, 4, 8, 12, (32 << 30) - 4]
+    for cb in cbs:
+        for t in (-3, -1, 0, 1, 2, 3, 5, 1000, 16383):
+            plain = ((cb >> 2) + t) >> 2
+            split = (cb >> 4) + ((((cb >> 2) & 3) + t) >> 2)
+            assert plain == split
+            assert -(1 << 31) <= (cb >> 4) < (1 << 31)  # the quad base itself fits the int32 it is kept in
