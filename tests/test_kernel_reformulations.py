@@ -7,7 +7,9 @@ result exactly (the GPU parity tests then check the kernels themselves):
   (build_tables.cu, normalize_warp) against the oracle's sequential greedy;
 * the range DP restricted to the end points that can still lie on a split into K non-empty
   ranges (build_tables.cu) against the oracle's full DP;
-* the decoder's ring-refill quad index, kept in 32 bits (decode.cu), against the plain formula.
+* the decoder's ring-refill quad index, kept in 32 bits (decode.cu), against the plain formula;
+* the encoder's bias trick for the renormalisation shift (encode.cu) against its definition;
+* the decoder's multiply-high field extractions (decode.cu) against plain shifts.
 """
 import numpy as np
 import pytest
@@ -147,3 +149,34 @@ def test_refill_quad_index_in_32_bits():
             split = (cb >> 4) + ((((cb >> 2) & 3) + t) >> 2)
             assert plain == split
             assert -(1 << 31) <= (cb >> 4) < (1 << 31)  # the quad base itself fits the int32 it is kept in
+
+
+def test_encoder_bias_trick_gives_the_defined_shift():
+    """The encoder takes nb = (X + bias) >> 16 with bias = ((R - a) << 16) - (f << (R - a)),
+    a = floor(log2 f); the oracle takes nb by its definition, the smallest shift with X >> nb < 2f.
+    Exhaustive over every count f and state X in [L, 2L) for L = 16 ... 4096."""
+    for R in range(4, 13):
+        L = 1 << R
+        X = np.arange(L, 2 * L, dtype=np.int64)
+        for f in range(1, L + 1):
+            a = f.bit_length() - 1
+            bias = ((R - a) << 16) - (f << (R - a))
+            nb = (X + bias) >> 16
+            assert np.all((X >> nb) < 2 * f) and np.all((X >> nb) >= f), (R, f)
+            # smallest such shift: one bit less would leave the state at or above 2f
+            assert np.all((nb == 0) | ((X >> np.maximum(nb - 1, 0)) >= 2 * f)), (R, f)
+
+
+def test_decoder_multiply_high_field_extraction():
+    """The decoder reads the fields of a table entry's second word with multiply-highs: y >> 8 as
+    mulhi(y, 2^24), (y >> 16) + a as mad.hi(y, 2^16, a), and the signed top byte added to the bit
+    position as mad.hi.s32(y, 2^8, p). Checked against the plain shifts on random words."""
+    rng = np.random.default_rng(11)
+    for y in [int(v) for v in rng.integers(0, 1 << 32, 5000, dtype=np.uint64)] + [0, 0xFFFFFFFF, 0x80000000, 0x7FFFFFFF]:
+        assert (y * (1 << 24)) >> 32 == y >> 8
+        a = int(rng.integers(0, 1 << 16))
+        assert ((y * (1 << 16)) >> 32) + a == (y >> 16) + a
+        ys = y - (1 << 32) if y >> 31 else y          # the word as a signed 32-bit value
+        p = int(rng.integers(0, 1 << 20))
+        top = (y >> 24) - 256 if (y >> 24) & 0x80 else (y >> 24)  # (int8)(y >> 24)
+        assert ((ys * 256) >> 32) + p == p + top
