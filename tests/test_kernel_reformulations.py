@@ -9,7 +9,9 @@ result exactly (the GPU parity tests then check the kernels themselves):
   ranges (build_tables.cu) against the oracle's full DP;
 * the decoder's ring-refill quad index, kept in 32 bits (decode.cu), against the plain formula;
 * the encoder's bias trick for the renormalisation shift (encode.cu) against its definition;
-* the decoder's multiply-high field extractions (decode.cu) against plain shifts.
+* the decoder's multiply-high field extractions (decode.cu) against plain shifts;
+* the decoder's per-slot table construction (modular inverse of the spread step, binary search,
+  rank count; decode.cu) against the oracle's tables.
 """
 import numpy as np
 import pytest
@@ -180,3 +182,44 @@ def test_decoder_multiply_high_field_extraction():
         p = int(rng.integers(0, 1 << 20))
         top = (y >> 24) - 256 if (y >> 24) & 0x80 else (y >> 24)  # (int8)(y >> 24)
         assert ((ys * 256) >> 32) + p == p + top
+
+
+def gpu_decode_slot(i, R, f, cumul):
+    """The decoder's table build computes each slot independently: the placement index tau of slot
+    i from the modular inverse of the spread step, the range of tau by binary search over the
+    cumulative counts, the slot's rank among its range's slots by counting placements below i."""
+    L = 1 << R
+    step = (L >> 1) + (L >> 3) + 3
+    inv = pow(step, -1, 1 << 32)
+    tau = (i * inv) & (L - 1)
+    a, b = 0, len(f) - 1
+    while a < b:
+        m = (a + b + 1) >> 1
+        if cumul[m] <= tau:
+            a = m
+        else:
+            b = m - 1
+    s = a
+    rank = sum(1 for u in range(cumul[s], cumul[s] + f[s]) if ((u * step) & (L - 1)) < i)
+    x = f[s] + rank
+    nb = R - (x.bit_length() - 1)
+    return s, nb, (x << nb) - L
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_decoder_slot_construction_matches_oracle_tables(orc, seed):
+    rng = np.random.default_rng(500 + seed)
+    R = int(rng.integers(4, 11))
+    L = 1 << R
+    K = int(rng.integers(1, min(L, 256) + 1))
+    f = np.zeros(K, np.int64)  # a random composition of L into K parts, empty ranges allowed
+    for u in rng.integers(0, K, L):
+        f[u] += 1
+    lo = np.sort(rng.choice(np.arange(1, 256), K - 1, replace=False)) if K > 1 else np.zeros(0, int)
+    lo = np.concatenate([[0], lo]).astype(np.uint16)
+    t = orc.tables(lo, f.astype(np.uint32), R)
+    cumul = np.concatenate([[0], np.cumsum(f)])[:K].tolist()
+    fl = f.tolist()
+    for i in range(L):
+        s, nb, nxt = gpu_decode_slot(i, R, fl, cumul)
+        assert (s, nb, nxt) == (t.dec_sym[i], t.dec_nb[i], t.dec_next[i]), (R, K, i)
