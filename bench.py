@@ -323,6 +323,12 @@ def cpu_baseline(x_dev, segs, p, budget_s, full_n):
     s, _ = oracle.encode(one, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], threads=cores)
     rc, _ = oracle.decode(s, threads=cores)
     dt1 = time.perf_counter() - t
+    # one thread, on a slice of the first segment (about a second of work)
+    m = min(one.size, max(p["chunk_symbols"], int(one.size * min(1.0, 1.0 / max(dt1 * cores, 1e-3)))))
+    t = time.perf_counter()
+    s1, _ = oracle.encode(one[:m], p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], threads=1)
+    oracle.decode(s1, threads=1)
+    one_thread_gbs = m / (time.perf_counter() - t) / 1e9
     k = max(1, min(len(segs), int(budget_s / max(dt1, 1e-3))))
     sample = [segs[i] for i in range(k)]
     xs = np.concatenate([x_dev[o:o + n].cpu().numpy() for o, n in sample])
@@ -340,7 +346,8 @@ def cpu_baseline(x_dev, segs, p, budget_s, full_n):
     nbytes = xs.size
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{k} of {len(segs)} segments ({nbytes} bytes): histogram+DP+tables+encode+decode, "
-                      f"{dt:.1f} s on {cores} host threads"}
+                      f"{dt:.1f} s on {cores} host threads",
+            "one_thread": {"value": one_thread_gbs, "unit": UNIT, "sample": f"first {m} bytes of segment 0"}}
 
 
 def run_regen(args):
