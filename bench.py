@@ -148,8 +148,8 @@ def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
     return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
 
 
-# DRAM bytes (read + write) per symbol of each kernel, from the ncu captures summarised in
-# profiles/<kernel>_kv_cache_1GiB.md (KV cache, K=16, L=128, C=4096, S=4), with the digest of the
+# DRAM bytes (read + write) per symbol of each kernel, from the ncu captures of that kernel on the
+# INT8 KV cache (K=16, L=128, C=4096, S=4), with the digest of the
 # kernel's source file (comments removed) at capture time: if the code has changed since, the figure
 # is stale and the bench reports traffic as null.
 MEASURED_TRAFFIC = {

@@ -62,6 +62,46 @@ EncWorkLayout enc_work_layout(uint64_t total_chunks, const shn_params* p) {
 
 }  // namespace
 
+namespace shn {
+
+int check_encode_args(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs, uint64_t* total_chunks,
+                      uint64_t* total_symbols) {
+  if (!params_ok(p)) return SHN_ERR_INVALID_ARG;
+  if (!segs_ok(h_segs, n_segs, total_chunks, total_symbols, p->chunk_symbols)) return SHN_ERR_INVALID_ARG;
+  // word offsets inside the payload are 32-bit: streams are limited to 16 GiB
+  if (shn_encode_bound(p, h_segs, n_segs) > (16ull << 30)) return SHN_ERR_INVALID_ARG;
+  return SHN_OK;
+}
+
+uint32_t fill_encode_batch(const shn_params& p, const shn_segment* h_segs, uint32_t n_segs, uint32_t s0,
+                           uint64_t& chunk, uint64_t& out_off, EncBatch& b) {
+  memset(&b, 0, sizeof(EncBatch));
+  uint64_t blocks = 0;
+  uint32_t si = s0;
+  for (; si < n_segs && b.n < (uint32_t)kSegBatch; ++si) {
+    const shn_segment& sg = h_segs[si];
+    const uint64_t nc = n_chunks(sg.length, p.chunk_symbols);
+    const uint32_t small = (nc <= kEncSmallMaxChunks) ? 1u : 0u;
+    if (b.n == 0) b.small = small;
+    else if (b.small != small) break;
+    const uint32_t i = b.n++;
+    b.offset[i] = sg.offset;
+    b.out_offset[i] = out_off;
+    b.length[i] = (uint32_t)sg.length;
+    b.first_chunk[i] = (uint32_t)chunk;
+    b.block_start[i] = (uint32_t)blocks;
+    b.seg_index[i] = si;
+    const uint64_t nt = small ? (uint64_t)kEncSmallThreads : (uint64_t)kEncBlockThreads;
+    blocks += (nc + nt - 1) / nt;
+    b.total_blocks = (uint32_t)blocks;
+    chunk += nc;
+    out_off += sg.length;
+  }
+  return si;
+}
+
+}  // namespace shn
+
 extern "C" {
 
 uint32_t shn_version(void) { return SHN_VERSION; }
@@ -151,15 +191,13 @@ int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params
 int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, const void* d_tables,
                const shn_params* p, void* d_work, size_t work_bytes, uint8_t* d_out, size_t out_capacity,
                uint64_t* d_out_bytes, void* stream) {
-  if (!params_ok(p)) return SHN_ERR_INVALID_ARG;
   uint64_t tc = 0, ts = 0;
-  if (!segs_ok(h_segs, n_segs, &tc, &ts, p->chunk_symbols)) return SHN_ERR_INVALID_ARG;
+  const int chk = check_encode_args(p, h_segs, n_segs, &tc, &ts);
+  if (chk != SHN_OK) return chk;
   if (!d_work || !d_out || !d_out_bytes || (n_segs > 0 && (!d_in || !d_tables))) return SHN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(d_out) & 15) || (reinterpret_cast<uintptr_t>(d_work) & 255) ||
       (reinterpret_cast<uintptr_t>(d_out_bytes) & 7) || (d_tables && (reinterpret_cast<uintptr_t>(d_tables) & 255)))
     return SHN_ERR_INVALID_ARG;
-  // word offsets inside the payload are 32-bit: streams are limited to 16 GiB
-  if (shn_encode_bound(p, h_segs, n_segs) > (16ull << 30)) return SHN_ERR_INVALID_ARG;
   const EncWorkLayout wl = enc_work_layout(tc, p);
   if (work_bytes < wl.total) return SHN_ERR_WORKSPACE;
   const bool single_pass = work_bytes >= wl.total_slots;
@@ -189,36 +227,14 @@ int shn_encode(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, 
   const shn_table* tables = static_cast<const shn_table*>(d_tables);
   if (cudaMemsetAsync(wb, 0, 8, s) != cudaSuccess) return SHN_ERR_CUDA;
 
-  // Segment batches (kernel parameters), built once and reused by every pass. A batch holds
-  // consecutive segments (the header pass indexes a contiguous chunk range per batch) of one kind:
-  // segments of at most kEncSmallMaxChunks chunks are coded by one-warp blocks with unreplicated
-  // tables, the others by kEncBlockThreads-thread blocks with lane-replicated tables.
+  // Segment batches (kernel parameters), built once and reused by every pass (fill_encode_batch:
+  // consecutive segments of one kind, so the header pass indexes a contiguous chunk range).
   std::vector<EncBatch> batches;
   {
-    uint64_t chunk = 0, out_off = 0, blocks = 0;
-    for (uint32_t si = 0; si < n_segs; ++si) {
-      const shn_segment& sg = h_segs[si];
-      const uint64_t nc = n_chunks(sg.length, p->chunk_symbols);
-      const uint32_t small = (nc <= kEncSmallMaxChunks) ? 1u : 0u;
-      if (batches.empty() || batches.back().n == (uint32_t)kSegBatch || batches.back().small != small) {
-        batches.emplace_back();
-        memset(&batches.back(), 0, sizeof(EncBatch));
-        batches.back().small = small;
-        blocks = 0;
-      }
-      EncBatch& b = batches.back();
-      const uint32_t i = b.n++;
-      b.offset[i] = sg.offset;
-      b.out_offset[i] = out_off;
-      b.length[i] = (uint32_t)sg.length;
-      b.first_chunk[i] = (uint32_t)chunk;
-      b.block_start[i] = (uint32_t)blocks;
-      b.seg_index[i] = si;
-      const uint64_t nt = small ? (uint64_t)kEncSmallThreads : (uint64_t)kEncBlockThreads;
-      blocks += (nc + nt - 1) / nt;
-      b.total_blocks = (uint32_t)blocks;
-      chunk += nc;
-      out_off += sg.length;
+    uint64_t chunk = 0, out_off = 0;
+    for (uint32_t si = 0; si < n_segs;) {
+      batches.emplace_back();
+      si = fill_encode_batch(*p, h_segs, n_segs, si, chunk, out_off, batches.back());
     }
   }
   // single pass: code every chunk into its slot (recording sizes); two passes: count sizes first

@@ -52,9 +52,6 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
-bool params_ok(const shn_params* p) { return shn_check_params(p) == SHN_OK; }
-
-
 }  // namespace
 
 extern "C" {
@@ -64,14 +61,11 @@ uint64_t shn_encode_static_max_chunks(void) { return kStaticMaxChunks; }
 int shn_encode_static(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_segs, const void* d_tables,
                       const shn_params* p, uint8_t* d_out, size_t out_capacity, uint64_t* d_out_bytes,
                       uint32_t* d_status, void* stream) {
-  if (!params_ok(p)) return SHN_ERR_INVALID_ARG;
-  if (n_segs > 0 && !h_segs) return SHN_ERR_INVALID_ARG;
+  // the checks shn_encode makes (parameters, segments, the 16 GiB stream limit), then the chunk
+  // count the static scratch holds
   uint64_t tc = 0, ts = 0;
-  for (uint32_t s = 0; s < n_segs; ++s) {
-    if (h_segs[s].length >= (1ull << 32)) return SHN_ERR_INVALID_ARG;
-    tc += n_chunks(h_segs[s].length, p->chunk_symbols);
-    ts += h_segs[s].length;
-  }
+  const int chk = check_encode_args(p, h_segs, n_segs, &tc, &ts);
+  if (chk != SHN_OK) return chk;
   if (tc > kStaticMaxChunks) return SHN_ERR_CAPACITY;
   if (!d_out || !d_out_bytes || !d_status || (n_segs > 0 && (!d_in || !d_tables))) return SHN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(d_out) & 15) || (reinterpret_cast<uintptr_t>(d_out_bytes) & 7) ||
@@ -107,32 +101,14 @@ int shn_encode_static(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n
   // (word counts by the size pass, offsets and block sums by the scan).
   if (cudaMemsetAsync(d_status, 0, sizeof(DeviceStatus), s) != cudaSuccess) return SHN_ERR_CUDA;
 
+  // shn_encode's two-pass launch sequence (sizes, scan, header and index, write in place) over the
+  // same segment batches; a batch is rebuilt on the stack for each pass instead of being kept.
   EncBatch b;
-  uint64_t chunk = 0, out_off = 0;
-  // the same launch sequence as shn_encode: sizes, scan, header/index, write; the batch
-  // parameters are rebuilt for each pass from h_segs
   for (int pass = 0; pass < 3; ++pass) {
-    chunk = 0;
-    out_off = 0;
+    uint64_t chunk = 0, out_off = 0;
     bool first = true;
-    for (uint32_t s0 = 0; s0 < n_segs; s0 += kSegBatch) {
-      memset(&b, 0, sizeof(b));
-      b.n = (n_segs - s0 < (uint32_t)kSegBatch) ? n_segs - s0 : (uint32_t)kSegBatch;
-      uint64_t blocks = 0;
-      for (uint32_t i = 0; i < b.n; ++i) {
-        const shn_segment& sg = h_segs[s0 + i];
-        b.offset[i] = sg.offset;
-        b.out_offset[i] = out_off;
-        b.length[i] = (uint32_t)sg.length;
-        b.first_chunk[i] = (uint32_t)chunk;
-        b.block_start[i] = (uint32_t)blocks;
-        b.seg_index[i] = s0 + i;
-        const uint64_t nc = n_chunks(sg.length, p->chunk_symbols);
-        blocks += (nc + kEncBlockThreads - 1) / kEncBlockThreads;
-        chunk += nc;
-        out_off += sg.length;
-      }
-      b.total_blocks = (uint32_t)blocks;
+    for (uint32_t s0 = 0; s0 < n_segs;) {
+      s0 = fill_encode_batch(*p, h_segs, n_segs, s0, chunk, out_off, b);
       cudaError_t e = cudaSuccess;
       if (pass == 0) e = launch_encode_sizes(d_in, b, tables, lay, w, 0, s);
       if (pass == 1) e = launch_encode_header(b, tables, lay, w, d_out, d_out_bytes, first, s);

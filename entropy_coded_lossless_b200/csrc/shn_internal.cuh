@@ -177,6 +177,20 @@ struct EncBatch {
   uint32_t seg_index[kSegBatch];   // segment / table index
 };
 
+// Host checks shared by shn_encode and shn_encode_static (capi.cu): parameters, segments (each
+// shorter than 2^32 symbols, fewer than 2^32 chunks in all) and the worst-case stream size, which
+// must stay within 16 GiB because chunk word offsets inside a payload are 32-bit. Returns SHN_OK or
+// SHN_ERR_INVALID_ARG; on success the chunk and symbol totals. No CUDA call.
+int check_encode_args(const shn_params* p, const shn_segment* h_segs, uint32_t n_segs, uint64_t* total_chunks,
+                      uint64_t* total_symbols);
+// Fills b with the encoder batch that starts at segment s0: up to kSegBatch consecutive segments of
+// one kind (segments of at most kEncSmallMaxChunks chunks are coded by one-warp blocks with
+// unreplicated tables, the others by kEncBlockThreads-thread blocks). chunk and out_off are the
+// global chunk index and output offset of segment s0, advanced past the batch. Returns the first
+// segment after the batch. Both encoder entry points build their launches with it.
+uint32_t fill_encode_batch(const shn_params& p, const shn_segment* h_segs, uint32_t n_segs, uint32_t s0,
+                           uint64_t& chunk, uint64_t& out_off, EncBatch& b);
+
 // Launch wrappers (defined in the .cu files; return a cudaError_t).
 cudaError_t launch_histogram(const uint8_t* d_in, const HistBatch& b, uint64_t* d_hist, int threads,
                              cudaStream_t s);

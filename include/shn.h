@@ -138,8 +138,8 @@ int shn_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params
  * Encode segments into one SHN1 stream (Shannonic §4.2, Algorithm 2: per value, s = rangeId[x],
  * emit the offset x - base[s] in nb[s] bits, emit the state-normalisation bits, move the state
  * through encTable). Chunks of C symbols are coded independently with S interleaved states.
- *  d_in          device input bytes; every segment offset must be 16-byte aligned with d_in
- *                16-byte aligned (SHN_ERR_INVALID_ARG otherwise).
+ *  d_in          device input bytes, any alignment (chunks whose bytes start on a 16-byte
+ *                boundary are read with 16-byte loads, the others byte by byte).
  *  h_segs        host, n_segs segments; segment s is coded with table s of d_tables.
  *  d_tables      device, n_segs records from shn_build_tables with the same params.
  *  d_work        device workspace of >= shn_encode_workspace_bytes_min(p, h_segs, n_segs) bytes,
@@ -253,12 +253,17 @@ int shn_decode_from_host(const uint8_t* const* h_streams, const size_t* stream_b
  * Limits and caveats:
  *  - more than SHN_STATIC_MAX_CHUNKS chunks in total returns SHN_ERR_CAPACITY (nothing enqueued);
  *  - the first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *    that device current; make that first call before any stream capture on that device;
+ *    that device current and keeps it for the life of the process; make that first call before any
+ *    stream capture on that device. A device reset (cudaDeviceReset, or the primary context
+ *    released and created again) may move the array: calls after one are not supported;
+ *  - it runs shn_encode's two-pass mode (each chunk is coded twice: once to size it, once to write
+ *    it in place), so it is slower than shn_encode with a single-pass workspace;
  *  - all calls share the one array: calls whose GPU work overlaps (different streams, or different
  *    host threads, without ordering between them) race and may produce corrupt streams. Order
  *    them on one stream or with events.
  * Never allocates: no cudaMalloc, cudaFree or allocating library routine is called.
- * Errors: as shn_encode (SHN_ERR_WORKSPACE cannot occur).
+ * Errors: as shn_encode, with the same host checks (including the 16 GiB stream limit, checked
+ *         before the chunk count); SHN_ERR_WORKSPACE cannot occur.
  */
 #define SHN_STATIC_MAX_CHUNKS 524288u
 uint64_t shn_encode_static_max_chunks(void);

@@ -102,3 +102,37 @@ def test_offload_queries_and_host_checks(lib, orc):
     assert call(stream, 10, 1000, 1 << 20) == shn.SHN_ERR_CORRUPT  # shorter than a header
     assert call(stream, stream.size, 999, 1 << 20) == shn.SHN_ERR_CAPACITY
     assert call(stream, stream.size, 1000, stream.size) == shn.SHN_ERR_WORKSPACE  # room for one stream only
+
+
+def test_static_encoder_host_checks(lib):
+    """shn_encode_static makes shn_encode's host checks before anything else, with no CUDA call:
+    a stream whose worst case passes 16 GiB (32-bit word offsets inside a payload) is refused even
+    when its chunk count fits the static scratch; so are a missing segment array and misaligned
+    pointers. The same oversized request is refused by shn_encode."""
+    import ctypes
+
+    L = shn.lib()
+    p = shn.CodecParams(16, 7, 65536, 4)
+    seg = (1 << 32) - 1
+    segs = [(i * seg, seg) for i in range(3)]  # about 196,608 chunks of 65,536 symbols
+    chunks = sum(-(-n // p.chunk_symbols) for _, n in segs)
+    assert chunks < shn.encode_static_max_chunks()
+    assert shn.encode_bound(p, segs) > (16 << 30)
+    arr = shn._segments(segs)
+    fake = 1 << 20  # a 256-byte aligned stand-in for device pointers: never dereferenced
+    pc = ctypes.byref(p.c())
+
+    def static(h_segs, n_segs, status=fake, out=fake):
+        return L.shn_encode_static(fake, h_segs, n_segs, fake, pc, out, 1 << 40, fake, status, None)
+
+    assert static(arr, 3) == shn.SHN_ERR_INVALID_ARG
+    assert L.shn_encode(fake, arr, 3, fake, pc, fake, 1 << 40, fake, 1 << 40, fake, None) == shn.SHN_ERR_INVALID_ARG
+    small = shn._segments([(0, 4096)])
+    assert static(None, 1) == shn.SHN_ERR_INVALID_ARG
+    assert static(small, 1, status=fake + 4) == shn.SHN_ERR_INVALID_ARG
+    assert static(small, 1, out=fake + 8) == shn.SHN_ERR_INVALID_ARG
+    # too many chunks for the static scratch (but a stream well within 16 GiB)
+    p128 = shn.CodecParams(16, 7, 128, 4)
+    many = shn._segments([(0, (shn.encode_static_max_chunks() + 1) * 128)])
+    assert L.shn_encode_static(fake, many, 1, fake, ctypes.byref(p128.c()), fake, 1 << 40, fake, fake,
+                               None) == shn.SHN_ERR_CAPACITY

@@ -64,6 +64,20 @@ def test_static_scratch_encoder_matches_workspace_encoder():
         assert torch.equal(out, expect)
 
 
+@pytest.mark.parametrize("K,R,C", [(16, 7, 65536), (256, 10, 4096)])
+def test_static_scratch_encoder_other_params(K, R, C):
+    """Long chunks (65,536 symbols) and plain tANS at L = 1024, each on two ragged segments: the
+    static path gives shn_encode's bytes for them too."""
+    p = shn.CodecParams(K, R, C, 4)
+    x = inputs.laplace_int8(300_007, 20.0, seed=K + R, device=DEV)
+    segs = [(0, 200_003), (200_003, 100_004)]
+    for _ in range(2):
+        codec, ref = _workspace_encoder(x, segs, p)
+        got, status = _static_encoder(x, segs, p, codec.tables)
+        assert status[0] == 0, status
+        assert torch.equal(got, ref)
+
+
 def test_static_scratch_encoder_rejects_too_many_chunks():
     p = shn.CodecParams(16, 7, 128, 4)
     n = (shn.encode_static_max_chunks() + 1) * 128
