@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused decode+dequantise measurement (kv)")
     ap.add_argument("--no-offload", action="store_true", help="skip the host offload/reload measurement (kv)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="kv: skip the other configurations (1, 2 with plain tANS, 4, and 5 at four entropies)")
     ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
     ap.add_argument("--entropy", type=float, default=5.3, choices=[2.0, 4.0, 5.3, 7.9], help="sweep workload")
     ap.add_argument("--K", type=int, default=None, help="override the workload's range count")
@@ -274,8 +276,9 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def stream_rate(stream_np, segs, p, hist):
-    """RP (payload bits/symbol), total bits/symbol and H from the stream and histograms (host, fp64)."""
+def stream_rate(stream_np, segs, p, hist, mask=None):
+    """RP (payload bits/symbol), total bits/symbol and H from the stream and histograms (host, fp64).
+    mask: segments to count (default all; the total then still covers the whole stream)."""
     hdr = np.frombuffer(stream_np[:64].tobytes(), dtype="<u8")
     index_off, payload_off = int(hdr[5]), int(hdr[6])
     n_segs = len(segs)
@@ -284,7 +287,8 @@ def stream_rate(stream_np, segs, p, hist):
     index = np.frombuffer(stream_np[index_off:index_off + 4 * total_chunks].tobytes(), dtype="<u4").astype(np.int64)
     words = np.frombuffer(stream_np[payload_off:].tobytes()[: (len(stream_np) - payload_off) // 4 * 4], dtype="<u4")
     payload_bits = 0
-    for s in range(n_segs):
+    sel = [s for s in range(n_segs) if mask is None or mask[s]]
+    for s in sel:
         first = int(descs[s, 7])
         nch = -(-segs[s][1] // p["chunk_symbols"])
         start_w = int(descs[s, 4] | (descs[s, 5] << 32)) // 4
@@ -297,10 +301,10 @@ def stream_rate(stream_np, segs, p, hist):
         T = 32 * (ends - 1) + hb  # sentinel position = bits before it
         T -= 32 * np.append(0, ends[:-1])
         payload_bits += int(T.sum()) - nch * p["states_per_chunk"] * p["log2L"]
-    n = sum(l for _, l in segs)
+    n = sum(segs[s][1] for s in sel)
     h = hist.reshape(-1, 256).astype(np.float64)
     ent = 0.0
-    for s in range(n_segs):
+    for s in sel:
         row = h[s]
         tot = row.sum()
         if tot > 0:
@@ -311,9 +315,74 @@ def stream_rate(stream_np, segs, p, hist):
     return {"payload": rp, "total": 8.0 * len(stream_np) / n, "entropy": H, "diff_pct": (rp - H) / H * 100.0}
 
 
-def cpu_baseline(x_dev, segs, p, budget_s, full_n):
+def theorem1_terms(stream_np, hist, R, mask=None):
+    """Shannonic §4, Theorem 1, per run: the code length closed form CL = H(P) + D_KL(P||Q) + sum_k P_k w_k
+    of every segment, from its histogram (host fp64) and the table record its stream carries (f, lo),
+    averaged over all symbols. P_k is the share of values in range k, Q_k = f_k / L the share of tANS
+    states it got, w_k = ceil(log2 |range k|) its offset width. With H the histogram entropy and
+    H(p|P) = H - H(P) the entropy left inside the ranges, the payload rate decomposes as
+        RP - H = D_KL(P||Q)                      (state-count quantisation, L finite)
+               + [sum_k P_k w_k - H(p|P)]        (fixed-width offsets, K ranges)
+               + [RP - CL]                       (the spread: tANS against its ideal Q)."""
+    hdr = np.frombuffer(stream_np[:64].tobytes(), dtype="<u4")
+    n_segs, K, tb = int(hdr[2]), int(hdr[3] & 0xFFFF), int(hdr[5])
+    L = 1 << R
+    h = hist.reshape(-1, 256).astype(np.float64)
+    rec0 = 64 + 32 * n_segs
+    acc = {"H": 0.0, "HP": 0.0, "DKL": 0.0, "offset": 0.0}
+    n_all = 0.0
+    for s in range(n_segs):
+        row = h[s]
+        n = row.sum()
+        if n == 0 or (mask is not None and not mask[s]):
+            continue
+        rec = stream_np[rec0 + tb * s: rec0 + tb * s + 3 * K]
+        f = np.frombuffer(rec[:2 * K].tobytes(), dtype="<u2").astype(np.float64)
+        lo = rec[2 * K:3 * K].astype(np.int64)
+        hi = np.append(lo[1:], 256)
+        Pk = np.array([row[a:b].sum() for a, b in zip(lo, hi)]) / n
+        w = np.array([int(b - a - 1).bit_length() for a, b in zip(lo, hi)], dtype=np.float64)
+        nz = Pk > 0
+        q = row[row > 0] / n
+        acc["H"] += n * float(-(q * np.log2(q)).sum())
+        acc["HP"] += n * float(-(Pk[nz] * np.log2(Pk[nz])).sum())
+        acc["DKL"] += n * float((Pk[nz] * np.log2(Pk[nz] / (f[nz] / L))).sum())
+        acc["offset"] += n * float((Pk * w).sum())
+        n_all += n
+    t = {k: v / n_all for k, v in acc.items()} if n_all else {k: 0.0 for k in acc}
+    t["H_given_P"] = t["H"] - t["HP"]
+    t["CL"] = t["HP"] + t["DKL"] + t["offset"]
+    t["offset_excess"] = t["offset"] - t["H_given_P"]
+    return {"H": t["H"], "H_P": t["HP"], "D_KL_P_Q": t["DKL"], "offset_bits": t["offset"],
+            "H_p_given_P": t["H_given_P"], "offset_excess": t["offset_excess"], "CL": t["CL"]}
+
+
+def rate_report(stream_np, segs, p, hist, mask=None):
+    """stream_rate plus the Theorem-1 terms and the spread's excess RP - CL."""
+    r = stream_rate(stream_np, segs, p, hist, mask)
+    t = theorem1_terms(stream_np, hist, p["log2L"], mask)
+    t["spread_excess"] = r["payload"] - t["CL"]
+    r["theorem1"] = t
+    return r
+
+
+def oracle_matches(x_dev, segs, p, gpu_stream_np, cores, stream=None):
+    """CPU-baseline leg: whether the oracle's SHN1 stream of the whole workload (all host threads)
+    is byte-identical to the GPU's. `stream` is the oracle stream if one was already made."""
+    import oracle
+
+    if stream is None:
+        xs = x_dev.view(torch.uint8).cpu().numpy()
+        stream, _ = oracle.encode(xs, p["K"], p["log2L"], p["states_per_chunk"], p["chunk_symbols"], segments=segs,
+                                  threads=cores)
+    return bool(stream.size == gpu_stream_np.size and np.array_equal(stream, gpu_stream_np))
+
+
+def cpu_baseline(x_dev, segs, p, budget_s, full_n, gpu_stream_np=None):
     """The CPU oracle as it stands (encode + decode, all host threads) on a bounded sample of the
-    same workload: whole segments, as many as fit the time budget (at least one)."""
+    same workload: whole segments, as many as fit the time budget (at least one). With the GPU's
+    stream of the whole workload it also reports whether the oracle's stream is byte-identical to
+    it (reusing the timed sample's stream when the sample is the whole workload)."""
     import oracle
 
     cores = oracle.cpu_count()
@@ -343,11 +412,17 @@ def cpu_baseline(x_dev, segs, p, budget_s, full_n):
     rc, y = oracle.decode(s, threads=cores)
     dt = time.perf_counter() - t
     assert rc == 0 and np.array_equal(y, xs.view(np.uint8))
+    del y
     nbytes = xs.size
-    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
-            "sample": f"{k} of {len(segs)} segments ({nbytes} bytes): histogram+DP+tables+encode+decode, "
-                      f"{dt:.1f} s on {cores} host threads",
-            "one_thread": {"value": one_thread_gbs, "unit": UNIT, "sample": f"first {m} bytes of segment 0"}}
+    out = {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+           "sample": f"{k} of {len(segs)} segments ({nbytes} bytes): histogram+DP+tables+encode+decode, "
+                     f"{dt:.1f} s on {cores} host threads",
+           "one_thread": {"value": one_thread_gbs, "unit": UNIT, "sample": f"first {m} bytes of segment 0"}}
+    if gpu_stream_np is not None:
+        whole = local == [(o, n) for o, n in segs]  # the sample is the workload, laid out the same way
+        del xs
+        out["oracle_identical"] = oracle_matches(x_dev, segs, p, gpu_stream_np, cores, stream=s if whole else None)
+    return out
 
 
 def run_regen(args):
@@ -439,6 +514,105 @@ def run_sweepgrid(args):
                       "unit": "points with K=16, L=128 within 1% of H", "n_gpus": 1, "higher_is_better": True,
                       "dtype": "u8", "data": "synthetic", "config": {"workload": "sweepgrid"}, "points": pts}),
           flush=True)
+
+
+def config_workloads(dev):
+    """The other configurations, in the order they are measured: (name, description, tensor,
+    segments, params, families or None). Drawn on the device from the same seeds the tests use."""
+    b53 = inputs.LAPLACE_B_FOR_ENTROPY[5.3]
+    base = dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4)
+    yield ("config1_laplace_65536", "65,536 i.i.d. truncated discrete Laplace (H = 5.3 bits), seed 0",
+           inputs.laplace_int8(65536, b53, seed=0, device=dev), None, dict(base), None)
+    w = inputs.weight_like_int8(seed=1, device=dev)
+    yield ("config2_weight_like_4096x1024", "weight-like [4096,1024], per-row absmax, 1% outliers x8, seed 1",
+           w, None, dict(base), None)
+    yield ("config2_plain_tans_L1024", "the same weight tensor, plain tANS: K = 256 identity ranges, L = 1024",
+           w, None, dict(base, K=256, log2L=10), None)
+    del w
+    x, segs, fam = inputs.activation_batch_int8(1024, 65536, seed=3, device=dev)
+    yield ("config4_activations_1024x65536", "1024 activation tensors x 65,536, per-tensor tables, seed 3",
+           x, segs, dict(base), fam)
+    del x
+    for H in (2.0, 4.0, 5.3, 7.9):
+        yield (f"config5_1GiB_H{H}", f"1 GiB truncated discrete Laplace, H = {H} bits, seed 4",
+               inputs.sweep_stream_int8(H, seed=4, device=dev), None, dict(base), None)
+
+
+def measure_config(shn, x, segs, p_dict, dev, stream, peak, reps=10, warmup=3):
+    """Median CUDA-event time of each stage over `reps` runs of histogram -> tables -> encode ->
+    decode (L2 flushed by a 256 MiB write before every run when the workload is below 256 MiB),
+    the rate report, and whether the round trip is exact. Returns (dict, GPU stream on the host)."""
+    p = shn.CodecParams(**p_dict)
+    codec = shn.Codec(segs, p, device=dev)
+    n = codec.n_symbols
+    out = torch.empty(n, dtype=torch.uint8, device=dev)
+    comp_cap = codec.stream_buf.numel()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if n < (1 << 28) else None
+    names = ("histogram", "build", "encode", "decode")
+    times = {k: [] for k in names}
+    for r in range(warmup + reps):
+        if flush is not None:
+            flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        codec.histogram(x)
+        ev[1].record(stream)
+        codec.build()
+        ev[2].record(stream)
+        codec.encode(x)
+        ev[3].record(stream)
+        codec.decode(codec.stream_buf, comp_cap, out)
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if r >= warmup:
+            for i, k in enumerate(names):
+                times[k].append(ev[i].elapsed_time(ev[i + 1]))
+    xb = x.view(torch.uint8).reshape(-1)
+    expect = torch.cat([xb[o:o + m] for o, m in segs])
+    ok = codec.status("enc")[0] == 0 and codec.status("dec")[0] == 0 and torch.equal(out, expect)
+    del expect
+    nbytes = int(codec.out_bytes.item())
+    stream_np = codec.stream_buf[:nbytes].cpu().numpy()
+    hist = codec.hist.cpu().numpy()
+    st = {k: statistics.median(v) for k, v in times.items()}
+    res = {"symbols": n, "segments": len(segs), "K": p.K, "L": 1 << p.log2L, "chunk_symbols": p.chunk_symbols,
+           "states_per_chunk": p.states_per_chunk, "stream_bytes": nbytes, "correct": bool(ok),
+           "ms": st, "step_ms": sum(st.values()),
+           "encode_gbs_int8": n / (st["encode"] * 1e-3) / 1e9, "decode_gbs_int8": n / (st["decode"] * 1e-3) / 1e9,
+           "encode_frac": (n + nbytes) / (st["encode"] * 1e-3) / 1e9 / peak,
+           "decode_frac": (n + nbytes) / (st["decode"] * 1e-3) / 1e9 / peak,
+           "timing": f"median of {reps} runs after {warmup} warm-up runs"
+                     + ("; L2 flushed before each run" if flush is not None else "; inputs larger than L2"),
+           "bits_per_symbol": rate_report(stream_np, segs, p_dict, hist)}
+    del codec, out, flush
+    return res, stream_np, hist
+
+
+def run_configs(shn, dev, stream, peak, cpu_check):
+    """Every configuration besides the headline one, measured on this GPU; with cpu_check the CPU
+    baseline leg also compares each GPU stream with the oracle's, byte for byte."""
+    res = {}
+    cores = None
+    for name, desc, x, segs, p_dict, fam in config_workloads(dev):
+        if segs is None:
+            segs = [(0, x.numel())]
+        r, stream_np, hist = measure_config(shn, x, segs, p_dict, dev, stream, peak)
+        r["workload"] = desc
+        if fam is not None:  # per family of activation tensor
+            names = ["laplace", "gaussian", "relu_gaussian"]
+            r["by_family"] = {names[f]: rate_report(stream_np, segs, p_dict, hist, mask=[v == f for v in fam])
+                              for f in range(3)}
+        if cpu_check:
+            import oracle
+
+            cores = cores or oracle.cpu_count()
+            t = time.perf_counter()
+            r["oracle_identical"] = oracle_matches(x, segs, p_dict, stream_np, cores)
+            r["oracle_check_s"] = time.perf_counter() - t
+        res[name] = r
+        del x, stream_np
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_reference(args):
@@ -598,7 +772,7 @@ def main():
     ok = est == 0 and dst == 0 and torch.equal(out, x.view(torch.uint8))
     nbytes = int(codec.out_bytes.item())
     stream_np = codec.stream_buf[:nbytes].cpu().numpy()
-    rate = stream_rate(stream_np, segs, p_dict, codec.hist.cpu().numpy())
+    rate = rate_report(stream_np, segs, p_dict, codec.hist.cpu().numpy())
     if args.workload == "int4":  # bits per weight as the pages count them: codes + one 32-bit scale per 64
         rate["total_with_group_scales"] = rate["total"] + 32 / 64
         rate["int4_alone_with_group_scales"] = 4 + 32 / 64
@@ -832,7 +1006,12 @@ def main():
             "e2e": e2e,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(x, segs, p_dict, args.cpu_sample_seconds, n)
+            line["cpu_baseline"] = cpu_baseline(x, segs, p_dict, args.cpu_sample_seconds, n, gpu_stream_np=stream_np)
+            line["oracle_identical"] = line["cpu_baseline"]["oracle_identical"]
+        if args.workload == "kv" and not args.segments and not args.no_configs:
+            del x, out, codec
+            torch.cuda.empty_cache()
+            line["configs"] = run_configs(shn, dev, stream, peak, cpu_check=not args.no_cpu_baseline and world == 1)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
