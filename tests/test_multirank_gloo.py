@@ -50,10 +50,10 @@ def _rank_main(rank, world, port, results):
 
 def test_two_gloo_ranks():
     world = 2
-    manager = mp.Manager()
+    ctx = mp.get_context("spawn")  # no fork: the test process may already run threads
+    manager = ctx.Manager()
     results = manager.dict()
     port = _free_port()
-    ctx = mp.get_context("spawn")
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, results)) for r in range(world)]
     for p in procs:
         p.start()
