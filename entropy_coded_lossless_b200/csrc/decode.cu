@@ -8,10 +8,14 @@
 // Tables. The decode table lives in shared memory as 8-byte entries
 //   .x = shared-window address of the next state's row (row base, including this thread's replica)
 //   .y = nb | w << 8 | base' << 16 | (-(nb + w) & 0xFF) << 24     (base' = range base ^ 0x80)
-// so one lookup plus two funnel shifts and one multiply-add give the next state's address. The
-// fields above bit 7 are written as multiply-highs (y >> s == mulhi(y, 2^(32-s)), and a signed
-// mulhi by 2^8 yields the negated field width); the compiler chooses shift or integer-multiply
-// instructions for them (forcing the multiply pipe for all of them measured slower). When a tile lies
+// so one lookup plus two funnel shifts and one multiply-add give the next state's address. Pipes:
+// the loop is bound by the ALU pipe (funnel shifts, byte permutes, compares; half rate on sm_100),
+// so work moves to the FMA pipe's integer multiply-add (also half rate, issued in parallel) where
+// it can: the next-state address, and the output value y + o * 2^16 (base' + offset in bits 16-23,
+// picked out by the byte permute that packs the output anyway). Multiply-highs are quarter rate
+// there; only the bit-position update keeps one (a signed mulhi by 2^8 adds the negated field
+// width from y's top byte). Per decoded value this is ~7.4 ALU and ~5.5 FMA-pipe instructions
+// (ncu pipe counts on the KV cache). When a tile lies
 // in one segment (the common case for large tensors) the table is stored interleaved
 // ([slot][replica], replica = lane & (copies - 1)): 16 copies up to L = 512, where an 8-byte load
 // is served per half-warp and the 16 lanes of a half-warp always hit 16 different bank pairs
@@ -286,8 +290,18 @@ struct ChunkCtx {
 };
 
 // Output sinks: where a chunk's decoded symbols go. Pieces are 16 consecutive output positions
-// (SHN1 format §6); put_pair/put receive raw bytes in their low 8 bits (junk above).
+// (SHN1 format §6). Each sink forms a symbol's value from its table word y (base' in bits 16-23)
+// and its offset o with val(y, o), and receives those values in put_pair/put.
 struct ByteSink {  // the INT8 tensor itself
+  // val = y + o * 2^16: the raw byte (base' + offset, mod 256) sits in bits 16-23, junk around it.
+  // One integer multiply-add (the multiplier is a runtime value, so it stays on the FMA pipe, which
+  // this ALU-bound loop has room on), where base' + o in the low byte would take ALU instructions.
+  uint32_t m16;  // 65536
+  __device__ __forceinline__ uint32_t val(uint32_t y, uint32_t o) const {
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(o), "r"(m16), "r"(y));
+    return d;
+  }
   uint8_t* out;
   uint8_t* dst;
   uint32_t stride;
@@ -301,13 +315,13 @@ struct ByteSink {  // the INT8 tensor itself
   __device__ __forceinline__ void begin_piece() {}
   // pp and i are loop indices of fully unrolled loops, so they fold to constants
   __device__ __forceinline__ void put_pair(int pp, uint32_t ba, uint32_t bb) {
-    const uint32_t pair = __byte_perm(ba, bb, 0x0040);  // bytes: ba.b0, bb.b0
+    const uint32_t pair = __byte_perm(ba, bb, 0x0062);  // bytes: ba.b2, bb.b2
     if ((pp & 1) == 0) ov[pp >> 1] = pair;
     else ov[pp >> 1] = __byte_perm(ov[pp >> 1], pair, 0x5410);
   }
-  __device__ __forceinline__ void put(int i, uint32_t b) {  // b's low byte into byte i % 4 of word i / 4
-    if ((i & 3) == 0) ov[i >> 2] = b;
-    else ov[i >> 2] = __byte_perm(ov[i >> 2], b, (i & 3) == 1 ? 0x3240u : (i & 3) == 2 ? 0x3410u : 0x4210u);
+  __device__ __forceinline__ void put(int i, uint32_t b) {  // b's byte 2 into byte i % 4 of word i / 4
+    if ((i & 3) == 0) ov[i >> 2] = __byte_perm(b, 0u, 0x0002);
+    else ov[i >> 2] = __byte_perm(ov[i >> 2], b, (i & 3) == 1 ? 0x3260u : (i & 3) == 2 ? 0x3610u : 0x6210u);
   }
   __device__ __forceinline__ void end_piece() {
     if (aligned) {
@@ -318,7 +332,7 @@ struct ByteSink {  // the INT8 tensor itself
     }
     dst += stride;
   }
-  __device__ __forceinline__ void put_tail(uint32_t i, uint32_t b) { dst[i] = (uint8_t)b; }
+  __device__ __forceinline__ void put_tail(uint32_t i, uint32_t b) { dst[i] = (uint8_t)(b >> 16); }
 };
 
 // bf16 dequantisation fused into the decode: value = bf16_rn(float(int8) * scale[pos >> gshift]),
@@ -326,6 +340,8 @@ struct ByteSink {  // the INT8 tensor itself
 // (groups are >= 16 positions and pieces start at multiples of 16), so there is one scale load per
 // piece, issued one piece ahead.
 struct Bf16Sink {
+  // val: the raw byte (base' + offset) in the low 8 bits, junk above
+  __device__ __forceinline__ uint32_t val(uint32_t y, uint32_t o) const { return add_shr16(y, o); }
   uint16_t* out;
   const float* scales;
   uint32_t gshift;
@@ -458,7 +474,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
         X[q] = E.x + r * (1u << SH);
         P = add_top_byte(E.y, P);
         advance();
-        sk.put(i, add_shr16(E.y, o));
+        sk.put(i, sk.val(E.y, o));
       }
     } else {
 #pragma unroll
@@ -471,7 +487,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
         const uint32_t wa = shr8(Ea.y);                            // low 5 bits: w
         const uint32_t oa = __funnelshift_l(Va, 0u, wa);           // offset: next w bits
         const uint32_t V2 = __funnelshift_l(0u, Va, wa);           // V << (nb + w)
-        const uint32_t ba = add_shr16(Ea.y, oa);                   // low byte: base' + offset
+        const uint32_t ba = sk.val(Ea.y, oa);                      // base' + offset
         X[qa] = Ea.x + ra * (1u << SH);
         P = add_top_byte(Ea.y, P);                                 // P -= nb + w
         const uint2 Eb = lds64(X[qb]);
@@ -479,7 +495,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
         const uint32_t Vb = __funnelshift_l(0u, V2, Eb.y);
         const uint32_t wb = shr8(Eb.y);
         const uint32_t ob = __funnelshift_l(Vb, 0u, wb);
-        const uint32_t bb = add_shr16(Eb.y, ob);
+        const uint32_t bb = sk.val(Eb.y, ob);
         X[qb] = Eb.x + rb * (1u << SH);
         P = add_top_byte(Eb.y, P);
         advance();
@@ -506,7 +522,7 @@ __device__ __forceinline__ bool decode_chunk(const ChunkCtx& c, uint32_t R, Sink
       x = E.x + r * (1u << SH);
       P = add_top_byte(E.y, P);
       advance();
-      sk.put_tail(i, add_shr16(E.y, o));
+      sk.put_tail(i, sk.val(E.y, o));
 #pragma unroll
       for (int k = 0; k < S; ++k)
         if (k == q) X[k] = x;
@@ -537,6 +553,7 @@ struct DecOut {
   const float* scales;
   uint32_t gshift;
   uint64_t n_scales;
+  uint32_t zero;  // 0, passed at run time so that multiplier operands stay opaque to the compiler
 };
 
 template <int S, bool BF16>
@@ -578,6 +595,7 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
       return decode_chunk<S, SH, PAIRS>(cc, h.R, sk);
     }
     ByteSink sk;
+    sk.m16 = 65536u | o.zero;
     sk.out = o.out;
     return decode_chunk<S, SH, PAIRS>(cc, h.R, sk);
   };
@@ -689,14 +707,14 @@ static cudaError_t launch_decode_mode(const uint8_t* d_comp, uint64_t comp_bytes
 
 cudaError_t launch_decode(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
                           uint8_t* d_out, uint64_t out_capacity, int sm_count, cudaStream_t s) {
-  const DecOut o{d_out, nullptr, 0u, 0ull};
+  const DecOut o{d_out, nullptr, 0u, 0ull, 0u};
   return launch_decode_mode<false>(d_comp, comp_bytes, p, st, o, out_capacity, sm_count, s);
 }
 
 cudaError_t launch_decode_bf16(const uint8_t* d_comp, uint64_t comp_bytes, const shn_params& p, DeviceStatus* st,
                                uint16_t* d_out, uint64_t out_elems, const float* d_scales, uint32_t log2_group,
                                uint64_t n_scales, int sm_count, cudaStream_t s) {
-  const DecOut o{reinterpret_cast<uint8_t*>(d_out), d_scales, log2_group, n_scales};
+  const DecOut o{reinterpret_cast<uint8_t*>(d_out), d_scales, log2_group, n_scales, 0u};
   return launch_decode_mode<true>(d_comp, comp_bytes, p, st, o, out_elems, sm_count, s);
 }
 
