@@ -52,6 +52,7 @@ def parse():
                     help="kv: skip the other configurations (1, 2 with plain tANS, 4, and 5 at four entropies)")
     ap.add_argument("--segments", type=int, default=0, help="kv workload: use only the first N segments")
     ap.add_argument("--entropy", type=float, default=5.3, choices=[2.0, 4.0, 5.3, 7.9], help="sweep workload")
+    ap.add_argument("--sweep-bytes", type=int, default=1 << 30, help="sweep workload: stream length (default 1 GiB)")
     ap.add_argument("--K", type=int, default=None, help="override the workload's range count")
     ap.add_argument("--log2L", type=int, default=None, help="override the workload's log2 state count")
     ap.add_argument("--chunk-symbols", type=int, default=None)
@@ -68,7 +69,7 @@ def apply_overrides(p, args):
             p[key] = val
 
 
-def workload(name, device, seed_offset=0, n_segments=0, entropy=5.3):
+def workload(name, device, seed_offset=0, n_segments=0, entropy=5.3, sweep_bytes=1 << 30):
     """(int8 tensor, segments, params dict, description)."""
     if name == "kv":
         segs = inputs.kv_cache_segments()
@@ -95,9 +96,9 @@ def workload(name, device, seed_offset=0, n_segments=0, entropy=5.3):
         x, segs, _ = inputs.activation_batch_int8(1024, 65536, seed=3 + seed_offset, device=device)
         desc = "1024 activation tensors x 65536 INT8 (per-tensor tables)"
     else:
-        x = inputs.sweep_stream_int8(entropy, seed=4 + seed_offset, device=device)
+        x = inputs.sweep_stream_int8(entropy, n=sweep_bytes, seed=4 + seed_offset, device=device)
         segs = [(0, x.numel())]
-        desc = f"1 GiB truncated discrete Laplace, H={entropy} bits"
+        desc = f"{sweep_bytes} bytes of truncated discrete Laplace, H={entropy} bits"
     return x, segs, dict(K=16, log2L=7, chunk_symbols=4096, states_per_chunk=4), desc
 
 
@@ -673,7 +674,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    x, segs, p, desc = workload(args.workload, "cpu", entropy=args.entropy)
+    x, segs, p, desc = workload(args.workload, "cpu", entropy=args.entropy, sweep_bytes=args.sweep_bytes)
     apply_overrides(p, args)
     import oracle
 
@@ -740,7 +741,7 @@ def main():
     from entropy_coded_lossless_b200 import shn
 
     x, segs, p_dict, desc = workload(args.workload, dev, seed_offset=rank, n_segments=args.segments,
-                                     entropy=args.entropy)
+                                     entropy=args.entropy, sweep_bytes=args.sweep_bytes)
     apply_overrides(p_dict, args)
     p = shn.CodecParams(**p_dict)
     codec = shn.Codec(segs, p, device=dev)

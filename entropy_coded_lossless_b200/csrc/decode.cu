@@ -1,9 +1,9 @@
 // decode.cu — chunk-parallel Shannonic/tANS decoder (Shannonic §4.2, decoding: the decode table
 // entry of the state gives the range s and its bit count, the offset o follows, x = base[s] + o).
 //
-// Work layout. A persistent grid of 256-thread blocks walks tiles of 256 consecutive chunks; each
-// thread decodes one chunk of C symbols with S interleaved states (SHN1 format §7), reading the chunk
-// backwards from its end sentinel.
+// Work layout. A persistent grid of 256-thread blocks, each taking a contiguous run of tiles of 256
+// consecutive chunks; each thread decodes one chunk of C symbols with S interleaved states (SHN1
+// format §7), reading the chunk backwards from its end sentinel.
 //
 // Tables. The decode table lives in shared memory as 8-byte entries
 //   .x = shared-window address of the next state's row (row base, including this thread's replica)
@@ -600,7 +600,13 @@ __global__ void __launch_bounds__(kDecThreads, DEC_MIN_BLOCKS) decode_kernel(con
     return decode_chunk<S, SH, PAIRS>(cc, h.R, sk);
   };
 
-  for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+  // Each block takes a contiguous run of tiles: consecutive tiles usually lie in one segment, so the
+  // replicated table is rebuilt only when the run crosses a segment boundary (a strided assignment
+  // rebuilt it for nearly every tile of a many-segment stream).
+  const uint64_t t_per = n_tiles / gridDim.x, t_rem = n_tiles % gridDim.x;
+  const uint64_t t_begin = blockIdx.x * t_per + min((uint64_t)blockIdx.x, t_rem);
+  const uint64_t t_end = t_begin + t_per + (blockIdx.x < t_rem ? 1u : 0u);
+  for (uint64_t tile = t_begin; tile < t_end; ++tile) {
     const uint64_t g0 = tile * kDecThreads;
     const uint64_t g_last = min(g0 + kDecThreads, h.total_chunks) - 1;
     const uint32_t sa = segment_of(descs, h.n_segs, g0), sb = segment_of(descs, h.n_segs, g_last);
