@@ -348,15 +348,21 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
     const uint32_t fs = S.f[s];
     const uint32_t o = u - S.lo[s];
     const uint32_t w = ceil_log2_width(S.lo[s + 1] - S.lo[s]);
+    // .x: bias + 2^22 in bits 0-22 (so that (X + .x) >> 16 = nb + 64, with the offset's bits from
+    //     bit 8 up), and the offset top-aligned in the w highest bits (a funnel shift of the state
+    //     bits into .x appends it below them);
+    // .y: w in bits 0-4 (a shift amount as it stands), bit 7 set for a byte whose range has no
+    //     states, encTable start + 4096 in bits 16-31.
+    const uint32_t off_top = w ? (o << (32u - w)) : 0u;
     uint2 e;
     if (fs == 0) {
-      e.x = 0u;  // nb = 0; enc index = X - L stays inside the table
-      e.y = o | (w << 8) | 0x8000u | ((4096u - L) << 16);  // absent-symbol flag
+      e.x = (1u << 22) + off_top;  // nb = 0; enc index = X - L stays inside the table
+      e.y = w | 0x80u | ((4096u - L) << 16);
     } else {
       const uint32_t a = 31u - __clz(fs);
       const uint32_t sh = (uint32_t)R - a;
-      e.x = (sh << 16) - (fs << sh);
-      e.y = o | (w << 8) | ((uint32_t)((int)S.cumul[s] - (int)fs + 4096) << 16);
+      e.x = (sh << 16) - (fs << sh) + (1u << 22) + off_top;
+      e.y = w | ((uint32_t)((int)S.cumul[s] - (int)fs + 4096) << 16);
     }
     reinterpret_cast<uint2*>(out->opaque + kOpaqueSymOffset)[bb] = e;
     out->f[tid] = (uint16_t)S.f[tid];

@@ -14,8 +14,11 @@
 // No device-wide spin waits; everything is ordered by the stream.
 //
 // Shared-memory tables. Each block codes chunks of one segment and keeps Algorithm 2's per-range
-// form in shared memory: sym[raw byte] = {bias, offset | w << 8 | (start + 4096) << 16}, with
-// bit 15 marking a byte absent from the table's histogram, and enc[L] (next state). A warp's 32
+// form in shared memory: sym[raw byte] = {bias + 2^22 with the offset in the top w bits,
+// w | (start + 4096) << 16} (bit 7 of .y marks a byte absent from the table's histogram), and
+// enc[L] (next state). The layout serves the ALU pipe, which bounds this loop: w sits where a shift
+// reads its amount, and one funnel shift of the state bits into .x appends the offset below them,
+// so a symbol's field costs one instruction instead of an extraction, a shift and an OR. A warp's 32
 // lookups use 32 unrelated indices, so both tables are stored lane-interleaved: sym 16 times
 // ([byte][16] x 8 bytes: an 8-byte load is served per half-warp, so the 16 lanes of a phase always
 // hit 16 distinct bank pairs) and enc in up to 8 KB of copies ([index][copies] x 4-byte slots; 16
@@ -73,19 +76,22 @@ struct Coder {
   uint32_t enc;      // this lane's column of enc, biased by -4096 rows (the +4096 in .y's start field)
   uint32_t enc_row;  // bytes per enc index (2 * copies)
   uint32_t L;
-  // Returns the symbol's fields (offset low, state bits above it); width = their total bit count.
-  // CHECK: accumulate .y into flags (bit 15 set for a byte absent from the table's histogram).
+  uint32_t absent;   // bit 7 set if a byte this thread staged has no states in the table
+  // Returns the symbol's fields (offset low, state bits above it); width = their total bit count in
+  // bits 0-5 (bit 5 clear), with junk above bit 5 that the bit counters ignore.
+  // CHECK: accumulate .y into flags (bit 7 set for a byte absent from the table's histogram).
+  // Every variable shift is a funnel shift, which uses its amount modulo 32: nb and w come with
+  // junk above bit 5 (see the entry layout), and no instruction is spent clearing it.
   template <bool CHECK>
   __device__ __forceinline__ uint32_t step(uint32_t b, uint32_t& X, uint32_t& width, uint32_t& flags) const {
     const uint2 e = lds64(sym + b * kSymRow);
-    const uint32_t nb = (X + e.x) >> 16;
-    const uint32_t q = X >> nb;
-    const uint32_t r = X - (q << nb);                   // the nb low state bits
-    const uint32_t w = __byte_perm(e.y, 0u, 0x4441u);  // offset width
+    const uint32_t nb = (X + e.x) >> 16;                 // nb + 64, offset bits from bit 8
+    const uint32_t q = __funnelshift_r(X, 0u, nb);       // X >> nb
+    const uint32_t r = X - __funnelshift_l(0u, q, nb);   // the nb low state bits
     X = lds_u16(enc + ((e.y >> 16) + q) * enc_row);
     if (CHECK) flags |= e.y;
-    width = w + nb;
-    return (r << w) | (e.y & 0xFFu);
+    width = e.y + nb;                                    // w + nb in bits 0-4
+    return __funnelshift_l(e.x, r, e.y);                 // (r << w) | offset (the top w bits of .x)
   }
 };
 
@@ -101,10 +107,12 @@ __device__ __forceinline__ bool load_coder(unsigned char* smem, const shn_table*
   uint2* s2 = reinterpret_cast<uint2*>(smem);
   unsigned char* e2 = smem + 256 * sym_copies * 8;
   bool narrow = true;
+  cd.absent = 0;
   for (uint32_t i = threadIdx.x; i < 256 * sym_copies; i += blockDim.x) {
     const uint2 e = sym[i / sym_copies];
     s2[i] = e;
-    narrow = narrow && R + ((e.y >> 8) & 0x7Fu) <= 16;  // bit 15 marks an absent byte, not width
+    narrow = narrow && R + (e.y & 31u) <= 16;
+    cd.absent |= e.y & 0x80u;
   }
   for (uint32_t i = threadIdx.x; i < L * copies; i += blockDim.x)
     *reinterpret_cast<uint16_t*>(e2 + i * kEncSlot) = enc[i / copies];
@@ -166,7 +174,7 @@ __device__ __forceinline__ void code_chunk(const CoderT& cd, const uint8_t* seg,
         uint32_t w1, w2;
         const uint32_t f1 = cd.template step<CHECK>(b1, st[r & (S - 1)], w1, flags);
         const uint32_t f2 = cd.template step<CHECK>(b2, st[(r - 1) & (S - 1)], w2, flags);
-        sink(f1 | (f2 << w1), w1 + w2);
+        sink(f1 + __funnelshift_l(0u, f2, w1), w1 + w2);  // w1 modulo 32; the two fields do not overlap
       }
     } else {
 #pragma unroll
@@ -200,7 +208,8 @@ __device__ __forceinline__ void code_chunk(const CoderT& cd, const uint8_t* seg,
 
 struct BitCounter {
   uint32_t bits = 0;  // a chunk has at most 65536 fields of <= 20 bits
-  __device__ __forceinline__ void operator()(uint32_t, uint32_t w) { bits += w; }
+  // w: bit count in bits 0-5 (at most 32), junk above
+  __device__ __forceinline__ void operator()(uint32_t, uint32_t w) { bits += w & 63u; }
   __device__ __forceinline__ void piece_done() {}
 };
 
@@ -210,15 +219,15 @@ struct RingWriter {
   uint32_t ring;         // shared address of this thread's row
   uint32_t* payload;     // stream payload, 16-byte aligned
   uint32_t wp, fp, end;  // next word to append, next word to store, end of this chunk (payload words)
-  uint32_t a0;           // the cnt (< 32) bits not yet in the ring
-  uint32_t cnt;
+  uint32_t a0;           // the bits not yet in the ring (cnt & 31 of them)
+  uint32_t cnt;          // bits 0-5: bits pending in a0 (< 32 between appends); junk above bit 5
   __device__ __forceinline__ uint32_t slot(uint32_t word) const { return ring + (word & (kRingWords - 1)) * 4u; }
-  // append the low n (<= 32) bits of v; the caller guarantees v < 2^n
+  // append the low (n & 63) <= 32 bits of v (junk in n above bit 5 is ignored); v < 2^(n & 63)
   __device__ __forceinline__ void operator()(uint32_t v, uint32_t n) {
-    a0 |= v << cnt;
-    const uint32_t over = __funnelshift_l(v, 0u, cnt);  // bits of v beyond position 32 (0 when cnt == 0)
-    cnt += n;
-    if (cnt >= 32) {
+    a0 += __funnelshift_l(0u, v, cnt);                  // v << (cnt & 31); a0 is zero from bit cnt & 31 up
+    const uint32_t over = __funnelshift_l(v, 0u, cnt);  // bits of v beyond position 32 (0 when cnt & 31 == 0)
+    cnt += n;                                            // bits 0-5: (cnt & 31) + (n & 63) <= 63, no carry out
+    if (cnt & 32u) {
       sts32(slot(wp), a0);
       ++wp;
       a0 = over;
@@ -236,7 +245,7 @@ struct RingWriter {
     }
   }
   __device__ __forceinline__ void finish() {
-    if (cnt > 0) {
+    if (cnt & 31u) {
       sts32(slot(wp), a0);
       ++wp;
     }
@@ -270,7 +279,7 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
   else code_chunk<S, false, true>(cd, in + b.offset[seg], geo, st, flags, bc);
   const uint64_t total = (uint64_t)bc.bits + (uint64_t)S * lay.R + 1;
   w.chunk_words[b.first_chunk[seg] + c] = (uint32_t)((total + 31) >> 5);
-  if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
+  if ((flags & 0x80u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, b.first_chunk[seg] + c);
 }
 
 // Writes every chunk's words. Two-pass mode (SLOTS = false): at the chunk's final place in the
@@ -288,6 +297,7 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
   const shn_table* t = tables + b.seg_index[seg];
   Coder<SMALL> cd;
   const bool narrow = __syncthreads_and(load_coder(esm, t, lay.R, cd));
+  const bool any_absent = __syncthreads_or(cd.absent != 0);  // block-uniform
   const uint32_t c = (blockIdx.x - b.block_start[seg]) * NT + threadIdx.x;
   const uint32_t len_seg = b.length[seg];
   if (c >= (uint32_t)n_chunks(len_seg, lay.C)) return;
@@ -310,15 +320,20 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
 #pragma unroll
   for (int q = 0; q < S; ++q) st[q] = cd.L;
   uint32_t flags = 0;
-  if (PAIRS || narrow) code_chunk<S, true, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
-  else code_chunk<S, false, SLOTS>(cd, in + b.offset[seg], geo, st, flags, rw);
+  if (SLOTS && any_absent) {  // the size pass is skipped: flag bytes absent from the table here
+    if (PAIRS || narrow) code_chunk<S, true, true>(cd, in + b.offset[seg], geo, st, flags, rw);
+    else code_chunk<S, false, true>(cd, in + b.offset[seg], geo, st, flags, rw);
+  } else {
+    if (PAIRS || narrow) code_chunk<S, true, false>(cd, in + b.offset[seg], geo, st, flags, rw);
+    else code_chunk<S, false, false>(cd, in + b.offset[seg], geo, st, flags, rw);
+  }
 #pragma unroll
   for (int q = 0; q < S; ++q) rw(st[q] - cd.L, lay.R);
   rw(1u, 1u);  // sentinel
   rw.finish();
   if (SLOTS) {
     w.chunk_words[g] = rw.wp;
-    if ((flags & 0x8000u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, (uint32_t)g);
+    if ((flags & 0x80u) || t->status != 0) report(w.status, SHN_ERR_INVALID_ARG, (uint32_t)g);
   }
 }
 

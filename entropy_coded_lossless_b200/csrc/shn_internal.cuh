@@ -60,10 +60,11 @@ __host__ __device__ inline ChunkGeo chunk_geo(uint64_t n, uint32_t C, uint32_t c
 }
 
 // ---- device table record (include/shn.h: shn_table) -----------------------------------------
-// opaque part: uint2 sym[256] for every raw byte b (u = b ^ 0x80):
-//   .x = bias[s]  (nb = (X + bias) >> 16),
-//   .y = offset | (w << 8) | (start[s] + 4096) << 16   with start[s] = cumul_s - f_s; bit 15 marks
-//        a byte whose range has no states (absent from the histogram the table was built from),
+// opaque part: uint2 sym[256] for every raw byte b (u = b ^ 0x80), range s, offset o = u - lo[s]:
+//   .x = bias[s] + 2^22 + (o << (32 - w))   (w > 0; bias[s] alone in bits 0-19): (X + .x) >> 16
+//        is nb + 64 with o's bits from bit 8 up, and the top w bits hold o,
+//   .y = w | (start[s] + 4096) << 16   with start[s] = cumul_s - f_s; bit 7 marks a byte whose range
+//        has no states (absent from the histogram the table was built from),
 // then uint16 enc[L] holding the next state L + slot.
 constexpr uint32_t kOpaqueSymOffset = 0;
 constexpr uint32_t kOpaqueEncOffset = 2048;
