@@ -291,7 +291,10 @@ __global__ void __launch_bounds__(SMALL ? kEncSmallThreads : kEncThreads) encode
     const uint8_t* __restrict__ in, const __grid_constant__ EncBatch b, const shn_table* __restrict__ tables,
     const EncodeLayout lay, EncodeWork w, uint8_t* __restrict__ out) {
   constexpr int NT = SMALL ? kEncSmallThreads : kEncThreads;
-  if (*(volatile uint32_t*)&w.status->status != 0) return;
+  // An error reported before this block started stops it. Another block of this launch may report
+  // one at any time, so one thread reads the word and the barrier gives every thread its answer:
+  // either all threads reach the barriers below or none does.
+  if (__syncthreads_or(threadIdx.x == 0 && *(volatile uint32_t*)&w.status->status != 0)) return;
   extern __shared__ __align__(16) unsigned char esm[];
   const int seg = block_segment(b);
   const shn_table* t = tables + b.seg_index[seg];
