@@ -7,12 +7,20 @@
 // tie-breaks, state-count allocation, spread) are SHN1 format §2-§5; this kernel must reproduce them
 // bit for bit, so it uses only integer arithmetic.
 //
-// Work is tiny (O(K·256²/2) min-plus steps per table) and latency-bound; one block of 512 threads
-// per table keeps everything in shared memory: the per-symbol cost factor (w << 24) - LG(count) of
-// every range [j, i) (a triangular 256x256 table of fixed-point log2 values), two DP rows and the
-// K x 257 argmin matrix. The DP layers are split over groups of 4 threads that each own one long and
-// one short end point, so every thread scans about the same number of candidate starts.
+// Work is small (O(K·256²/2) min-plus steps per table) and latency-bound, so a table is built by a
+// cluster of G blocks (G = 1, 2, 4 or 8: the launch takes the largest G that still gives every
+// block its own SM). The DP's end points i = 1..256 are paired as (256 - g, g + 1), g = 0..127,
+// which together have 257 candidate starts whatever g; a group of 4G threads of cluster block r
+// owns pair g = group * G + r. A block keeps the per-symbol cost factor (w << 24) - LG(count) of
+// the ranges [j, i) ending at its own end points (257 entries per pair) and a copy of the two DP
+// rows; after each layer every group writes its two new cells into every block's row copy and its
+// argmins into block 0, through distributed shared memory, and the cluster meets at a barrier.
+// Block 0 then backtracks and builds the rest of the table alone (state counts, spread, tables).
+#include <cooperative_groups.h>
+
 #include "shn_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace shn {
 
@@ -29,9 +37,12 @@ __global__ void __launch_bounds__(256) lg_table_kernel() {
   for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < kLgTableSize; c += gridDim.x * blockDim.x)
     g_lg_table[c] = lg_fixed(c);
 }
-constexpr int kPairs = 256 * 257 / 2;  // ranges [j, i), 0 <= j < i <= 256
 
 __device__ __forceinline__ uint32_t ceil_log2_width(uint32_t m) { return m <= 1 ? 0u : 32u - __clz(m - 1u); }
+
+// Words per end-point pair of the cost-factor table in a block of a G-block cluster: room for both
+// rows (257 words) after row ib's shift of up to 31 words, rounded to 4G modulo 32.
+__host__ __device__ constexpr int build_stride(int G) { return 4 * G == 32 ? 288 : 288 + 4 * G; }
 
 struct BuildShared {
   uint32_t pre[257];       // prefix sums of the histogram (total < 2^32)
@@ -139,22 +150,39 @@ __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L
   }
 }
 
-__global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsigned long long* __restrict__ hist_all,
-                                                                     shn_params p, shn_table* __restrict__ tables_out,
-                                                                     uint32_t use_lg_table) {
+// G blocks per table (launched as clusters of G when G > 1).
+template <int G>
+__global__ void __launch_bounds__(kBuildThreads)
+    build_tables_kernel(const unsigned long long* __restrict__ hist_all, shn_params p,
+                        shn_table* __restrict__ tables_out, uint32_t use_lg_table) {
+  constexpr int T = 4 * G;                 // threads per end-point pair (a power of two that divides 32)
+  constexpr int P = 128 / G;               // end-point pairs per block
+  constexpr int kStride = build_stride(G);  // words per pair's cost factors
+  static_assert(P * T == kBuildThreads, "every thread of a block works on one pair");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BuildShared& S = *reinterpret_cast<BuildShared*>(smem_raw);
-  uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));          // kPairs cost factors
-  uint8_t* arg = reinterpret_cast<uint8_t*>(lgc + kPairs);                               // K x 257
+  uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));  // P x kStride cost factors
+  uint8_t* arg = reinterpret_cast<uint8_t*>(lgc + P * kStride);                    // K x 257 (used in block 0)
+  // G = 1 is an ordinary launch: block barriers and this block's own shared memory
+  cg::cluster_group cluster = cg::this_cluster();
+  const uint32_t rank = G > 1 ? cluster.block_rank() : 0u;
+  auto cluster_sync = [&]() {
+    if constexpr (G > 1) cluster.sync();
+    else __syncthreads();
+  };
+  auto in_block = [&](auto* ptr, int r) {
+    if constexpr (G > 1) return cluster.map_shared_rank(ptr, r);
+    else return ptr;
+  };
 
   const int tid = threadIdx.x;
   const int K = (int)p.K;
   const int R = (int)p.log2L;
   const uint32_t L = 1u << R;
-  const unsigned long long* hist = hist_all + (size_t)blockIdx.x * 256;
-  shn_table* out = tables_out + blockIdx.x;
+  const unsigned long long* hist = hist_all + (size_t)(blockIdx.x / G) * 256;
+  shn_table* out = tables_out + blockIdx.x / G;
 
-  // ---- prefix sums and the 2^32 bound --------------------------------------------------------
+  // ---- prefix sums and the 2^32 bound (every block of the cluster, from the same counts) ------
   if (tid < 32) {  // warp 0: lane l sums counts 8l .. 8l+7, then a shuffle scan over the lanes
     unsigned long long v[8], acc = 0;
 #pragma unroll
@@ -177,13 +205,16 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
       S.pre[0] = 0;
       S.status = incl >= (1ull << 32) ? (uint32_t)SHN_ERR_INVALID_ARG : 0u;
       S.cost = 0;
-      out->n = incl;
+      if (rank == 0) out->n = incl;
     }
   }
-  for (uint32_t f = tid; f <= L; f += kBuildThreads) S.lgf[f] = lg_fixed(f);
+  if (rank == 0)
+    for (uint32_t f = tid; f <= L; f += kBuildThreads) S.lgf[f] = lg_fixed(f);
   __syncthreads();
+  // Every block reaches the same decision from the same counts, so a cluster either runs all of its
+  // barriers below or none.
   if (S.status != 0) {
-    if (tid == 0) {
+    if (rank == 0 && tid == 0) {
       out->K = K;
       out->log2L = R;
       out->status = S.status;
@@ -193,6 +224,7 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
 
   // ---- range selection (SHN1 format §3) ---------------------------------------------------------
   if (K == 256) {
+    if (rank != 0) return;
     if (tid < 256) {
       S.lo[tid] = tid;
       const uint32_t n = S.pre[tid + 1] - S.pre[tid];
@@ -200,57 +232,58 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
       atomicAdd(reinterpret_cast<unsigned long long*>(&S.cost), 0ull - (unsigned long long)n * lg_fixed(n));
     }
   } else {
-    // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30; warp w
-    // fills the rows i = w+1, w+17, ... (about the same number of pairs per warp)
+    const int grp = tid / T, lane = tid % T;  // a group is T consecutive lanes of one warp
+    const int g = grp * G + (int)rank;
+    const int ia = 256 - g, ib = g + 1;
+    // Row ia, then row ib from word ia + (g mod 32) of the pair's block: with a stride of T mod 32
+    // words, both rows of the groups of one warp start T banks apart, so the T lanes of each group
+    // read T consecutive banks that no other group of the warp uses.
+    uint32_t* lg_a = lgc + grp * kStride;
+    uint32_t* lg_b = lg_a + ia + (g & 31);
+    // per-symbol cost of range [j, i) in units of 2^-24 bit: w << 24 - LG(count), |.| < 2^30
     const bool lookup = use_lg_table && S.pre[256] < kLgTableSize;  // every count of the segment is < 2^17
-    for (int i = 1 + (tid >> 5); i <= 256; i += kBuildThreads / 32) {
-      const uint32_t pi = S.pre[i];
-      uint32_t* row = lgc + i * (i - 1) / 2;
-      for (int j = tid & 31; j < i; j += 32)
-        row[j] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) -
-                            (int32_t)(lookup ? __ldg(g_lg_table + (pi - S.pre[j])) : lg_fixed(pi - S.pre[j])));
+    for (int e = lane; e < 257; e += T) {
+      const int i = e < ia ? ia : ib, j = e < ia ? e : e - ia;
+      const uint32_t c = S.pre[i] - S.pre[j];
+      (e < ia ? lg_a : lg_b)[j] = (uint32_t)((int32_t)(ceil_log2_width((uint32_t)(i - j)) << 24) -
+                                             (int32_t)(lookup ? __ldg(g_lg_table + c) : lg_fixed(c)));
     }
     for (int i = tid; i <= 256; i += kBuildThreads) S.drow[0][i] = (i == 0) ? 0 : LLONG_MAX;
-    __syncthreads();
-    // Balanced min-plus layers: group g of 4 threads owns the end points ia = 256 - g and ib = g + 1
-    // (together ~257 candidate starts whatever g), and its threads take every 4th candidate of the
-    // concatenated lists. Each thread scans its candidates in ascending j with a strict <, and the
-    // group reduction prefers the smaller value, then the smaller j: the smallest j wins ties.
+    cluster_sync();  // every block has started and initialised its rows before any remote write
+    uint8_t* arg0 = in_block(arg, 0);
+    // Layer k: the group's lanes take every T-th candidate start in ascending j with a strict <, and
+    // the group reduction prefers the smaller value, then the smaller j: the smallest j wins ties.
     // Only end points i <= 256 - (K - k) can lie on a split into K non-empty ranges (the K - k ranges
     // still to come need a symbol each), and every cell that does reads only such cells of the layer
     // before; the cells above that band are never read, so they are not computed (at K = 256 the
     // band is the single split into identity ranges).
-    const int r4 = tid & 3;
-    const int ia = 256 - (tid >> 2), ib = (tid >> 2) + 1;
+    const uint32_t pa = S.pre[ia], pb = S.pre[ib];
     for (int k = 1; k <= K; ++k) {
       const long long* prev = S.drow[(k - 1) & 1];
-      long long* cur = S.drow[k & 1];
       const int imax = 256 - (K - k);
       const int na = (ia >= k && ia <= imax) ? ((k == 1) ? 1 : ia - k + 1) : 0;  // j = k-1 .. (k == 1 ? 0 : i-1)
       const int nb = (ib >= k && ib <= imax) ? ((k == 1) ? 1 : ib - k + 1) : 0;
       long long best_a = LLONG_MAX, best_b = LLONG_MAX;
       int bj_a = 0x7fffffff, bj_b = 0x7fffffff;
-      const uint32_t pa = S.pre[ia], pb = S.pre[ib];
-      const int base_a = ia * (ia - 1) / 2, base_b = ib * (ib - 1) / 2;
-      // Cost(j, i-1) = c * (w << 24) - c * LG(c) = c * lgc[pair]; each thread takes every 4th start
-      for (int t = r4; t < na; t += 4) {
+      // Cost(j, i-1) = c * (w << 24) - c * LG(c) = c * lg[j]
+      for (int t = lane; t < na; t += T) {
         const int j = (k - 1) + t;
-        const long long v = prev[j] + (long long)(pa - S.pre[j]) * (long long)(int32_t)lgc[base_a + j];
+        const long long v = prev[j] + (long long)(pa - S.pre[j]) * (long long)(int32_t)lg_a[j];
         if (v < best_a) {
           best_a = v;
           bj_a = j;
         }
       }
-      for (int t = r4; t < nb; t += 4) {
+      for (int t = lane; t < nb; t += T) {
         const int j = (k - 1) + t;
-        const long long v = prev[j] + (long long)(pb - S.pre[j]) * (long long)(int32_t)lgc[base_b + j];
+        const long long v = prev[j] + (long long)(pb - S.pre[j]) * (long long)(int32_t)lg_b[j];
         if (v < best_b) {
           best_b = v;
           bj_b = j;
         }
       }
 #pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
+      for (int o = 1; o < T; o <<= 1) {
         const long long oa = __shfl_xor_sync(0xffffffffu, best_a, o);
         const int oja = __shfl_xor_sync(0xffffffffu, bj_a, o);
         if (oa < best_a || (oa == best_a && oja < bj_a)) {
@@ -264,18 +297,17 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
           bj_b = ojb;
         }
       }
-      if (r4 == 0 && na > 0) {
-        cur[ia] = best_a;
-        arg[(size_t)(k - 1) * 257 + ia] = (uint8_t)bj_a;
-      }
-      if (r4 == 1 && nb > 0) {
-        cur[ib] = best_b;
-        arg[(size_t)(k - 1) * 257 + ib] = (uint8_t)bj_b;
-      }
-      if (tid == 0) cur[0] = LLONG_MAX;
-      if (tid < 257 && tid < k) cur[tid] = LLONG_MAX;
-      __syncthreads();
+      // lanes 0..G-1 write cell ia into blocks 0..G-1, lanes G..2G-1 cell ib; lanes 2G and 2G+1 the
+      // argmins (into block 0)
+      long long* cur = S.drow[k & 1];
+      if (lane < G && na > 0) in_block(cur, lane)[ia] = best_a;
+      if (lane >= G && lane < 2 * G && nb > 0) in_block(cur, lane - G)[ib] = best_b;
+      if (lane == 2 * G && na > 0) arg0[(size_t)(k - 1) * 257 + ia] = (uint8_t)bj_a;
+      if (lane == 2 * G + 1 && nb > 0) arg0[(size_t)(k - 1) * 257 + ib] = (uint8_t)bj_b;
+      if (tid < k) cur[tid] = LLONG_MAX;  // cells below the band, in this block's copy (no one else writes them)
+      cluster_sync();
     }
+    if (rank != 0) return;  // no block reads another's shared memory after the last barrier
     if (tid == 0) {
       S.cost = S.drow[K & 1][256];
       int ii = 256;
@@ -379,20 +411,44 @@ __global__ void __launch_bounds__(kBuildThreads) build_tables_kernel(const unsig
   }
 }
 
+template <int G>
+static cudaError_t launch_build_g(const uint64_t* d_hist, uint32_t n_tables, const shn_params& p, shn_table* d_tables,
+                                 uint32_t use_table, cudaStream_t s) {
+  const size_t smem = sizeof(BuildShared) + sizeof(uint32_t) * (128 / G) * build_stride(G) + (size_t)p.K * 257;
+  cudaError_t e = cudaFuncSetAttribute(build_tables_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_tables * G, 1, 1);
+  cfg.blockDim = dim3(kBuildThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = G > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, build_tables_kernel<G>, reinterpret_cast<const unsigned long long*>(d_hist), p,
+                            d_tables, use_table);
+}
+
 cudaError_t launch_build_tables(const uint64_t* d_hist, uint32_t n_tables, const shn_params& p, shn_table* d_tables,
                                 cudaStream_t s) {
   if (n_tables == 0) return cudaSuccess;
-  const size_t smem = sizeof(BuildShared) + sizeof(uint32_t) * kPairs + (size_t)p.K * 257;
-  cudaError_t e = cudaFuncSetAttribute(build_tables_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const uint32_t use_table = n_tables >= kLgTableMinTables ? 1u : 0u;
   if (use_table) {
     lg_table_kernel<<<128, 256, 0, s>>>();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
-  build_tables_kernel<<<n_tables, kBuildThreads, smem, s>>>(reinterpret_cast<const unsigned long long*>(d_hist), p,
-                                                            d_tables, use_table);
-  return cudaGetLastError();
+  // the largest cluster that still gives each block an SM of its own; large batches of tables are
+  // throughput-bound and keep one block per table (the fewest instructions per table)
+  const uint64_t sms = (uint64_t)sm_count_for_launch();
+  if ((uint64_t)n_tables * 8 <= sms) return launch_build_g<8>(d_hist, n_tables, p, d_tables, use_table, s);
+  if ((uint64_t)n_tables * 4 <= sms) return launch_build_g<4>(d_hist, n_tables, p, d_tables, use_table, s);
+  if ((uint64_t)n_tables * 2 <= sms) return launch_build_g<2>(d_hist, n_tables, p, d_tables, use_table, s);
+  return launch_build_g<1>(d_hist, n_tables, p, d_tables, use_table, s);
 }
 
 }  // namespace shn
