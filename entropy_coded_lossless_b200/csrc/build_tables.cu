@@ -57,9 +57,16 @@ struct BuildShared {
   long long cost;
 };
 
-// Greedy state allocation on one warp (SHN1 format §4): every range with a count starts with one
-// state; each further state goes to the range with the largest N_k * (LG(f_k + 1) - LG(f_k)),
-// ties to the smallest k. kPer ranges per lane (K <= 32 * kPer).
+// Scratch of the threshold allocation, placed over the DP's cost factors (dead by then).
+struct NormScratch {
+  unsigned long long red64[kBuildThreads / 32];  // block reductions
+  uint32_t red32[kBuildThreads / 32];
+  uint32_t ties[256];                            // per range: gains equal to the threshold, then those taken
+};
+
+// Greedy state allocation on one warp (SHN1 format §4), one state per step, for L <= 128 (K <= 128):
+// every range with a count starts with one state; each further state goes to the range with the
+// largest N_k * (LG(f_k + 1) - LG(f_k)), ties to the smallest k. kPer ranges per lane (K <= 32 * kPer).
 template <int kPer>
 __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L, int tid) {
   unsigned long long N[kPer];
@@ -150,6 +157,81 @@ __device__ __forceinline__ void normalize_warp(BuildShared& S, int K, uint32_t L
   }
 }
 
+// State counts (SHN1 format §4): every range with a count starts with one state; each further state
+// goes to the range with the largest gain N_k * (LG(f_k + 1) - LG(f_k)), ties to the smallest k.
+// Each range's gains form a non-increasing sequence in f_k (LG's fixed-point differences never grow
+// for f <= 4096), so the M = L - nonzero states that greedy hands out one by one are the first M
+// elements (k, f) in the order (gain down, k up, f up): every element whose gain is above the M-th
+// largest gain v, then the elements equal to v in range order. The block finds v by bisection on the
+// gain, each thread counting its range's elements above a trial value (thread k holds range k).
+// Used from L = 256 up, where it takes fewer block-wide rounds (about 56) than the greedy has steps.
+__device__ void normalize_block(BuildShared& S, NormScratch& Z, int K, uint32_t L, int tid) {
+  const int lane = tid & 31, wid = tid >> 5;
+  const unsigned long long N = tid < K ? (unsigned long long)(S.pre[S.lo[tid + 1]] - S.pre[S.lo[tid]]) : 0ull;
+  auto sum_u32 = [&](uint32_t v) -> uint32_t {  // block-wide, every thread gets the sum
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) Z.red32[wid] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int i = 0; i < kBuildThreads / 32; ++i) t += Z.red32[i];
+    __syncthreads();
+    return t;
+  };
+  const uint32_t nonzero = sum_u32(N > 0 ? 1u : 0u);
+  if (nonzero == 0) {  // an empty segment: all states on range 0
+    if (tid < K) S.f[tid] = tid == 0 ? L : 0u;
+    return;
+  }
+  const uint32_t M = L - nonzero;  // K <= L is checked on the host, so nonzero <= L
+  // gain of the (f + 1)-th state, f = 1 .. L - 1
+  auto gain = [&](uint32_t f) -> unsigned long long { return N * (unsigned long long)(S.lgf[f + 1] - S.lgf[f]); };
+  // number of this range's elements with gain > tau: the largest f in [1, L-1] with gain(f) > tau, or
+  // 0. Started from f ~ N 2^24 / (tau ln 2) (the gains are close to N 2^24 / (f ln 2)) and corrected
+  // in unit steps, which is exact because the gains never increase with f.
+  auto count_gt = [&](unsigned long long tau) -> uint32_t {
+    if (N == 0) return 0;
+    const float est = (float)N * 24204406.32f / fmaxf((float)tau, 1.0f);  // 2^24 / ln 2
+    uint32_t f = est >= (float)(L - 1) ? L - 1 : (uint32_t)est;
+    while (f + 1 <= L - 1 && gain(f + 1) > tau) ++f;
+    while (f >= 1 && gain(f) <= tau) --f;
+    return f;
+  };
+  uint32_t f = N > 0 ? 1u : 0u;
+  if (M > 0) {
+    unsigned long long hi = N > 0 ? gain(1) : 0ull;  // no element is above the largest first gain
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    if (lane == 0) Z.red64[wid] = hi;
+    __syncthreads();
+    hi = 0;
+#pragma unroll
+    for (int i = 0; i < kBuildThreads / 32; ++i) hi = max(hi, Z.red64[i]);
+    unsigned long long lo = 0;  // all L - 1 elements of every counted range are above 0, and M <= that
+    while (hi - lo > 1) {       // invariant: at least M elements above lo, fewer than M above hi
+      const unsigned long long mid = lo + ((hi - lo) >> 1);
+      if (sum_u32(count_gt(mid)) >= M) lo = mid;
+      else hi = mid;
+    }
+    const unsigned long long v = hi;  // the M-th largest gain
+    const uint32_t above = count_gt(v);
+    const uint32_t r = M - sum_u32(above);  // elements equal to v that are taken, in range order
+    if (tid < K) Z.ties[tid] = count_gt(v - 1) - above;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t seen = 0;
+      for (int k = 0; k < K; ++k) {
+        const uint32_t e = Z.ties[k];
+        Z.ties[k] = seen >= r ? 0u : min(e, r - seen);
+        seen += e;
+      }
+    }
+    __syncthreads();
+    if (N > 0) f = 1 + above + Z.ties[tid];
+  }
+  if (tid < K) S.f[tid] = f;  // S.f[K..255] were zeroed by the caller
+}
+
 // G blocks per table (launched as clusters of G when G > 1).
 template <int G>
 __global__ void __launch_bounds__(kBuildThreads)
@@ -159,6 +241,7 @@ __global__ void __launch_bounds__(kBuildThreads)
   constexpr int P = 128 / G;               // end-point pairs per block
   constexpr int kStride = build_stride(G);  // words per pair's cost factors
   static_assert(P * T == kBuildThreads, "every thread of a block works on one pair");
+  static_assert(sizeof(NormScratch) <= sizeof(uint32_t) * P * kStride, "the allocation scratch fits the cost table");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BuildShared& S = *reinterpret_cast<BuildShared*>(smem_raw);
   uint32_t* lgc = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BuildShared));  // P x kStride cost factors
@@ -323,12 +406,14 @@ __global__ void __launch_bounds__(kBuildThreads)
   if (tid < 256) S.f[tid] = 0;
   __syncthreads();
 
-  // ---- state counts (SHN1 format §4): one warp, greedy with smallest-k tie-break ---------------
-  if (tid < 32) {
+  // ---- state counts (SHN1 format §4): the greedy one state per step on one warp at L <= 128, its
+  // result by a threshold on the gains at larger L --------------------------------------------------
+  if (L >= 256) {
+    normalize_block(S, *reinterpret_cast<NormScratch*>(lgc), K, L, tid);
+  } else if (tid < 32) {
     if (K <= 32) normalize_warp<1>(S, K, L, tid);
     else if (K <= 64) normalize_warp<2>(S, K, L, tid);
-    else if (K <= 128) normalize_warp<4>(S, K, L, tid);
-    else normalize_warp<8>(S, K, L, tid);
+    else normalize_warp<4>(S, K, L, tid);
   }
   __syncthreads();
   if (tid == 0) {

@@ -4,7 +4,11 @@ against the oracle on random inputs, so that each reformulation is shown to give
 result exactly (the GPU parity tests then check the kernels themselves):
 
 * the greedy state allocation with cached per-range gains and a per-lane tournament
-  (build_tables.cu, normalize_warp) against the oracle's sequential greedy;
+  (build_tables.cu, normalize_warp, used at L <= 128) against the oracle's sequential greedy;
+* the same allocation computed as a threshold on the gains (build_tables.cu, normalize_block, used
+  from L = 256: bisection on the M-th largest gain, per-range counts from an estimate corrected in
+  unit steps, ties in range order) against the oracle's sequential greedy, and the premise that
+  makes it exact: the fixed-point LG differences never increase;
 * the range DP restricted to the end points that can still lie on a split into K non-empty
   ranges (build_tables.cu) against the oracle's full DP;
 * the decoder's ring-refill quad index, kept in 32 bits (decode.cu), against the plain formula;
@@ -65,9 +69,10 @@ def tournament_greedy(N, R, lgf):
 
 @pytest.mark.parametrize("seed", range(40))
 def test_tournament_greedy_matches_oracle(orc, seed):
+    """The kernel uses this form at L <= 128 (so K <= 128)."""
     rng = np.random.default_rng(seed)
-    K = int(rng.choice([1, 3, 16, 31, 33, 64, 100, 129, 200, 256]))
-    R = int(rng.integers(max(4, int(np.ceil(np.log2(K)))), 11))
+    K = int(rng.choice([1, 3, 16, 31, 33, 64, 100, 128]))
+    R = int(rng.integers(max(4, int(np.ceil(np.log2(K)))), 8))
     top = min(1 << int(rng.choice([6, 20, 31])), (1 << 32) // (K + 1))  # the total stays below 2^32
     pool = rng.integers(1, top, 4)  # few distinct counts: many ties
     N = rng.choice(np.concatenate([[0, 0, 1], pool]), K).astype(np.uint64)
@@ -75,6 +80,88 @@ def test_tournament_greedy_matches_oracle(orc, seed):
         N[(1 << R):] = 0
     expect = orc.normalize(N, R)
     got = tournament_greedy(N, R, lg_table(orc, 1 << R))
+    assert list(expect) == got
+
+
+def threshold_allocation(N, R, lgf):
+    """The kernel's form: every range with a count starts with one state; the M = L - nonzero further
+    states are the M first elements (k, f) in the order (gain down, k up, f up), gain =
+    N_k (LG(f+1) - LG(f)) for f = 1 .. L-1: all elements above the M-th largest gain v, found by
+    bisection on the gain, then the elements equal to v in range order. A range's count above a
+    trial value starts from N 2^24 / (tau ln 2) and is corrected in unit steps."""
+    K = len(N)
+    L = 1 << R
+    n = [int(v) for v in N]
+    nonzero = sum(1 for v in n if v > 0)
+    if nonzero == 0:
+        return [L] + [0] * (K - 1)
+    M = L - nonzero
+
+    def gain(k, f):
+        return n[k] * (lgf[f + 1] - lgf[f])
+
+    def count_gt(k, tau):
+        if n[k] == 0:
+            return 0
+        est = float(np.float32(n[k]) * np.float32(24204406.32) / np.float32(max(tau, 1)))
+        f = L - 1 if est >= L - 1 else int(est)
+        while f + 1 <= L - 1 and gain(k, f + 1) > tau:
+            f += 1
+        while f >= 1 and gain(k, f) <= tau:
+            f -= 1
+        return f
+
+    f = [1 if v > 0 else 0 for v in n]
+    if M > 0:
+        lo, hi = 0, max(gain(k, 1) for k in range(K) if n[k] > 0)
+        while hi - lo > 1:
+            mid = lo + (hi - lo) // 2
+            if sum(count_gt(k, mid) for k in range(K)) >= M:
+                lo = mid
+            else:
+                hi = mid
+        v = hi
+        above = [count_gt(k, v) for k in range(K)]
+        r = M - sum(above)
+        seen = 0
+        for k in range(K):
+            e = count_gt(k, v - 1) - above[k]
+            take = 0 if seen >= r else min(e, r - seen)
+            seen += e
+            if n[k] > 0:
+                f[k] = 1 + above[k] + take
+    return f
+
+
+def test_lg_differences_never_increase(orc):
+    """The premise of the threshold form: LG(f+1) - LG(f) is non-increasing for f = 1 .. 4096, so
+    every range's gain sequence is non-increasing (the greedy then takes each range's elements in
+    order, and its picks are a prefix of one global order)."""
+    lgf = lg_table(orc, 4096)
+    d = [lgf[f + 1] - lgf[f] for f in range(1, 4097)]
+    assert all(d[i + 1] <= d[i] for i in range(len(d) - 1))
+    assert any(d[i + 1] == d[i] for i in range(len(d) - 1))  # equal neighbours exist: ties within a range
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_threshold_allocation_matches_oracle(orc, seed):
+    rng = np.random.default_rng(seed)
+    K = int(rng.choice([1, 3, 16, 31, 33, 64, 100, 129, 200, 256]))
+    R = int(rng.integers(max(4, int(np.ceil(np.log2(K)))), 13))
+    top = min(1 << int(rng.choice([6, 20, 31])), (1 << 32) // (K + 1))  # the total stays below 2^32
+    mode = seed % 3
+    if mode == 0:  # few distinct counts: many ties between ranges
+        pool = rng.integers(1, top, 4)
+        N = rng.choice(np.concatenate([[0, 0, 1], pool]), K).astype(np.uint64)
+    elif mode == 1:
+        N = rng.integers(0, top, K).astype(np.uint64)
+    else:  # one dominant range: thousands of states on it, where neighbouring gains can be equal
+        N = rng.integers(0, 4, K).astype(np.uint64)
+        N[rng.integers(0, K)] = top
+    if int((N > 0).sum()) > (1 << R):
+        N[(1 << R):] = 0
+    expect = orc.normalize(N, R)
+    got = threshold_allocation(N, R, lg_table(orc, 1 << R))
     assert list(expect) == got
 
 
