@@ -472,7 +472,7 @@ def run_regen(args):
     for name, n, seg, paper_s in (("ResNet-50-sized weights", 51_000_000, 12_750_000, 0.052),
                                   ("Gemma-2-9B-sized weights", 8_700_000_000, 21_750_000, 15.4)):
         x = inputs.laplace_int8(n, 7.258, seed=7, device=dev)
-        segs = [(o, min(seg, n - o)) for o in range(0, n, seg)]
+        segs = shn.Segments([(o, min(seg, n - o)) for o in range(0, n, seg)])  # marshalled once
         codec_hist = torch.zeros(len(segs) * 256, dtype=torch.int64, device=dev)
         tables = shn.empty_aligned(len(segs) * shn.TABLE_BYTES, dev)
         stream = torch.cuda.current_stream()
@@ -948,8 +948,10 @@ def main():
         copy_stream = torch.cuda.Stream(dev)
         placed = {}
 
+        segs_c = shn.Segments(segs)  # marshalled once
+
         def do_offload():  # blocks until the last batch is encoded; the copies finish on copy_stream
-            placed["offs"], placed["sizes"] = shn.shn_offload(x, segs, ends, p, owork, h_all, stream, copy_stream)
+            placed["offs"], placed["sizes"] = shn.shn_offload(x, segs_c, ends, p, owork, h_all, stream, copy_stream)
             stream.wait_stream(copy_stream)
 
         do_offload()

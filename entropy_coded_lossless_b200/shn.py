@@ -115,11 +115,26 @@ def _check(code: int, what: str):
         raise ShnError(code, what)
 
 
+class Segments:
+    """A segment list marshalled once into the C array the ABI takes (reused on every call)."""
+
+    def __init__(self, segments):
+        self.pairs = [(int(o), int(n)) for o, n in segments]
+        self.arr = (Segment * max(1, len(self.pairs)))()
+        for i, (o, n) in enumerate(self.pairs):
+            self.arr[i].offset, self.arr[i].length = o, n
+
+    def __len__(self):
+        return len(self.pairs)
+
+    def __iter__(self):
+        return iter(self.pairs)
+
+
 def _segments(segments):
-    arr = (Segment * max(1, len(segments)))()
-    for i, (o, n) in enumerate(segments):
-        arr[i].offset, arr[i].length = int(o), int(n)
-    return arr
+    if isinstance(segments, Segments):
+        return segments.arr
+    return Segments(segments).arr
 
 
 def _dev(t: torch.Tensor, name: str, host_ok: bool = False) -> int:
@@ -296,7 +311,7 @@ class Codec:
         """single_pass: allocate the encoder workspace that lets every chunk be coded once into its
         own slot (about the stream bound); otherwise the minimal one (two-pass encoder)."""
         self.p = p
-        self.segments = [(int(o), int(n)) for o, n in segments]
+        self.segments = Segments(segments)  # marshalled once: the calls below reuse the C array
         self.device = torch.device(device)
         ns = len(self.segments)
         self.hist = torch.zeros(max(1, ns) * 256, dtype=torch.int64, device=self.device)
