@@ -166,6 +166,26 @@ def test_params_and_ragged_segments(orc, K, R, S, C):
     check_parity(orc, x, segs, shn.CodecParams(K, R, C, S))
 
 
+@pytest.mark.parametrize("n_tables", [1, 18, 19, 37, 38, 74, 75, 160])
+def test_table_build_cluster_sizes(orc, n_tables):
+    """The table build runs a cluster of 8, 4 or 2 blocks per table, or one block, by how many
+    tables the launch has (the largest cluster that still gives every block an SM: on 148 SMs the
+    switches fall between 18 and 19, 37 and 38, 74 and 75 tables); every table record and the
+    stream must equal the oracle's whichever is taken. Segments of different lengths and
+    entropies, two of them beyond 2^17 symbols (LG computed, not looked up)."""
+    rng = np.random.default_rng(n_tables)
+    lens = rng.integers(2_000, 40_000, n_tables)
+    lens[0], lens[-1] = 150_000, 200_000
+    parts = [inputs.laplace_int8(int(n), float(rng.choice([0.8, 3.0, 7.0, 40.0])), seed=1000 + i).numpy()
+             for i, n in enumerate(lens)]
+    x = np.concatenate(parts)
+    ends = np.cumsum(lens)
+    segs = [(int(e - n), int(n)) for e, n in zip(ends, lens)]
+    check_parity(orc, x, segs, shn.CodecParams(16, 7, 1024, 4))
+    if n_tables in (19, 38):  # the threshold allocation (L >= 256) under a cluster of 4 and of 2
+        check_parity(orc, x, segs, shn.CodecParams(32, 9, 1024, 4))
+
+
 def test_degenerate_inputs(orc):
     p = shn.CodecParams(16, 7, 1024, 4)
     single = np.full(5000, -7, np.int8)
