@@ -1,4 +1,4 @@
-// build_tables.cu — per-segment range selection and tANS tables, one block per table.
+// build_tables.cu — per-segment range selection and tANS tables, a cluster of blocks per table.
 //
 // Shannonic §4.1 (preprocessing): partition the 256-value alphabet into K contiguous ranges by the
 // DP C[i,k] = min_{j<i} { C[j,k-1] + Cost(j,i-1) } with backtracking from C[256,K]; derive the

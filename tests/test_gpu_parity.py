@@ -182,7 +182,7 @@ def test_table_build_cluster_sizes(orc, n_tables):
     ends = np.cumsum(lens)
     segs = [(int(e - n), int(n)) for e, n in zip(ends, lens)]
     check_parity(orc, x, segs, shn.CodecParams(16, 7, 1024, 4))
-    if n_tables in (19, 38):  # the threshold allocation (L >= 256) under a cluster of 4 and of 2
+    if n_tables in (19, 38, 160):  # the threshold allocation (L >= 256): clusters of 4 and 2, one block
         check_parity(orc, x, segs, shn.CodecParams(32, 9, 1024, 4))
 
 
