@@ -514,6 +514,13 @@ static cudaError_t launch_build_g(const uint64_t* d_hist, uint32_t n_tables, con
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = G > 1 ? 1 : 0;
+  if constexpr (G > 1) {  // a device that cannot place such a cluster builds with one block per table
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, build_tables_kernel<G>, &cfg) != cudaSuccess || clusters < 1) {
+      (void)cudaGetLastError();
+      return launch_build_g<1>(d_hist, n_tables, p, d_tables, use_table, s);
+    }
+  }
   return cudaLaunchKernelEx(&cfg, build_tables_kernel<G>, reinterpret_cast<const unsigned long long*>(d_hist), p,
                             d_tables, use_table);
 }
