@@ -175,7 +175,7 @@ MEASURED_TRAFFIC = {
     "build_tables_kernel": {
         "bytes_per_symbol": 0.0003,
         "source": "build_tables.cu",
-        "sha256_prefix": "6ace10f1f1be3945"
+        "sha256_prefix": "687e0c81ec448e3a"
     },
     "encode_compact_kernel": {
         "bytes_per_symbol": 1.7616,
