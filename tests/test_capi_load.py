@@ -136,3 +136,19 @@ def test_static_encoder_host_checks(lib):
     many = shn._segments([(0, (shn.encode_static_max_chunks() + 1) * 128)])
     assert L.shn_encode_static(fake, many, 1, fake, ctypes.byref(p128.c()), fake, 1 << 40, fake, fake,
                                None) == shn.SHN_ERR_CAPACITY
+
+
+def test_segment_list_marshalled_once(lib):
+    """shn.Segments holds the C array a call takes; the binding passes it through unchanged (a
+    codec reuses it on every call), and its sizes agree with a plain list's."""
+    pairs = [(0, 5000), (5000, 0), (12_345, 77), (1 << 33, 4096 * 3 + 1)]
+    sg = shn.Segments(pairs)
+    assert len(sg) == len(pairs) and list(sg) == pairs
+    arr = shn._segments(sg)
+    assert arr is sg.arr and shn._segments(sg) is arr
+    assert [(arr[i].offset, arr[i].length) for i in range(len(pairs))] == pairs
+    p = shn.CodecParams(16, 7, 4096, 4)
+    assert shn.encode_bound(p, sg) == shn.encode_bound(p, pairs) > 0
+    assert shn.encode_workspace_bytes(p, sg) == shn.encode_workspace_bytes(p, pairs) > 0
+    empty = shn.Segments([])
+    assert len(empty) == 0 and len(shn._segments(empty)) == 1  # the C array is never empty
