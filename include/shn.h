@@ -124,7 +124,8 @@ int shn_histogram(const uint8_t* d_in, const shn_segment* h_segs, uint32_t n_seg
  * Range selection and tANS tables for each histogram (Shannonic §4.1: DP range selection
  * C[i,k] = min_{j<i} C[j,k-1] + Cost(j,i-1) with backtracking from C[256,K]; per-range base,
  * offset width, encTable start and bias; rangeId[256]; an L-state tANS table from the range
- * probabilities). Exact rules: SHN1 format §2-§5. One CUDA block per table.
+ * probabilities). Exact rules: SHN1 format §2-§5. Each table is built by a cluster of 2, 4 or 8
+ * blocks when the launch leaves SMs free for that, otherwise by one block (same records).
  *  d_hist    device, n_tables*256 uint64 (as written by shn_histogram).
  *  d_tables  device, n_tables*shn_table_bytes(p) bytes, 256-byte aligned; fully overwritten.
  * A histogram whose total is >= 2^32 gets status SHN_ERR_INVALID_ARG in its record (and makes
