@@ -163,9 +163,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "4ba1ae6f524ade66"
     },
     "encode_write_kernel": {
-        "bytes_per_symbol": 2.0241,
+        "bytes_per_symbol": 2.0253,
         "source": "encode.cu",
-        "sha256_prefix": "19b89331d5155e21"
+        "sha256_prefix": "d5136af6dad60ad2"
     },
     "histogram_kernel": {
         "bytes_per_symbol": 1.0125,
@@ -178,9 +178,9 @@ MEASURED_TRAFFIC = {
         "sha256_prefix": "687e0c81ec448e3a"
     },
     "encode_compact_kernel": {
-        "bytes_per_symbol": 1.7616,
+        "bytes_per_symbol": 1.7239,
         "source": "encode.cu",
-        "sha256_prefix": "19b89331d5155e21"
+        "sha256_prefix": "d5136af6dad60ad2"
     }
 }
 
